@@ -1,0 +1,332 @@
+"""Seeded synthetic inputs for one MiniMax-H3 transformer block.
+
+This module is shared by the CPU oracle (``oracle/``), the tests and the
+benchmark. It holds no arithmetic of the block itself: only the dimensions,
+the packed row layouts (modality tag, timestep index and (t, h, w) rotary
+position per row) and seeded random tensors of the stated distributions.
+
+Where the layouts come from:
+
+* "MiniMaxH3Transformer3DModel" (diffusers API page), introduction: one packed
+  1-D sequence of text, conditioning image/video, audio and target-video rows;
+  padding rows carry tag -1 and form their own attention document.
+* Same page, ``forward`` parameters: per-row ``token_tags``,
+  ``timestep_indices`` and ``position_ids`` of shape (seq_len, 3).
+* Same page, constructor parameters: hidden 5376, 56 heads of 128, ffn 14336,
+  rope_theta 1e4, norm_eps and qk_norm_eps 1e-5.
+* The t2va geometry (124 frames at 1344x768 -> a 31 x 24 x 42 latent grid of
+  2x2 patches) follows the diffusers MiniMax-H3 pipeline page, memory section.
+
+Values: x ~ N(0, 1); every weight ~ N(0, 1/fan_in); modulation table ~
+N(0, 0.1^2); per-head norm gains 1 + N(0, 0.1^2). Everything is drawn in fp32 with
+``numpy.random.default_rng(seed)`` and rounded to bf16 where the block stores
+bf16 (x, weights, gains). The modulation table stays fp32.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field, replace
+
+import numpy as np
+import torch
+
+TAG_PAD = -1
+
+
+@dataclass(frozen=True)
+class Dims:
+    hidden: int
+    heads: int
+    head_dim: int
+    ffn: int
+    n_tags: int
+    n_t: int
+    rope_pairs: tuple  # (t, h, w) rotary pairs; the remaining head_dim/2 pairs pass through
+    rope_theta: float = 10000.0
+    norm_eps: float = 1e-5
+    qk_norm_eps: float = 1e-5
+    quant: int = 0  # 0: bf16 linears, 1: rotated W8A8 linears
+
+    @property
+    def hd(self) -> int:
+        return self.heads * self.head_dim
+
+
+TINY = Dims(hidden=256, heads=6, head_dim=64, ffn=768, n_tags=4, n_t=2, rope_pairs=(8, 12, 12))
+REAL = Dims(hidden=5376, heads=56, head_dim=128, ffn=14336, n_tags=4, n_t=2, rope_pairs=(16, 24, 24))
+
+
+@dataclass
+class Layout:
+    """Per-row structure of one packed sequence."""
+    name: str
+    tag: np.ndarray    # int32 [N], -1 = padding
+    tidx: np.ndarray   # int32 [N]
+    pos: np.ndarray    # int32 [N, 3] (t, h, w)
+    segments: list = field(default_factory=list)  # (label, start, count)
+
+    @property
+    def n(self) -> int:
+        return int(self.tag.shape[0])
+
+    @property
+    def n_valid(self) -> int:
+        return int((self.tag != TAG_PAD).sum())
+
+    @property
+    def n_pad(self) -> int:
+        return self.n - self.n_valid
+
+
+class _Builder:
+    """Appends row segments in sequence order."""
+
+    def __init__(self, name):
+        self.name = name
+        self.tags, self.tidx, self.pos, self.segments = [], [], [], []
+        self.n = 0
+
+    def add(self, label, tag, tidx, pos):
+        pos = np.asarray(pos, dtype=np.int32).reshape(-1, 3)
+        k = pos.shape[0]
+        tidx = np.broadcast_to(np.asarray(tidx, dtype=np.int32), (k,))
+        self.tags.append(np.full(k, tag, dtype=np.int32))
+        self.tidx.append(np.array(tidx, dtype=np.int32))
+        self.pos.append(pos)
+        self.segments.append((label, self.n, k))
+        self.n += k
+
+    def build(self) -> Layout:
+        return Layout(self.name, np.concatenate(self.tags), np.concatenate(self.tidx),
+                      np.concatenate(self.pos), self.segments)
+
+
+def text_positions(n):
+    i = np.arange(n, dtype=np.int32)
+    return np.stack([i, i, i], axis=1)
+
+
+def audio_positions(n, t0=0):
+    j = np.arange(n, dtype=np.int32) + t0
+    z = np.zeros(n, dtype=np.int32)
+    return np.stack([j, z, z], axis=1)
+
+
+def grid_positions(t, h, w, t0=0):
+    tt, hh, ww = np.meshgrid(np.arange(t) + t0, np.arange(h), np.arange(w), indexing="ij")
+    return np.stack([tt.ravel(), hh.ravel(), ww.ravel()], axis=1).astype(np.int32)
+
+
+def pad_positions(n):
+    return np.zeros((n, 3), dtype=np.int32)
+
+
+def _round_up(n, m):
+    return (n + m - 1) // m * m
+
+
+# Tag numbering used by every measured layout: 0 text, 1 conditioning
+# (image / video references), 2 audio, 3 target video. A tag is only an index
+# into the modulation table.
+TAG_TEXT, TAG_COND, TAG_AUDIO, TAG_VIDEO = 0, 1, 2, 3
+
+
+def layout_tiny(seed=0) -> Layout:
+    """320 rows: 64 text, 32 audio, 192 video on a (3, 8, 8) grid, 32 padding.
+    Per-row timestep index drawn uniformly from {0, 1}."""
+    b = _Builder("tiny_320")
+    b.add("text", TAG_TEXT, 0, text_positions(64))
+    b.add("audio", TAG_AUDIO, 0, audio_positions(32))
+    b.add("video", TAG_VIDEO, 0, grid_positions(3, 8, 8))
+    b.add("pad", TAG_PAD, 0, pad_positions(32))
+    lay = b.build()
+    rng = np.random.default_rng(seed + 1000)
+    lay.tidx = rng.integers(0, 2, size=lay.n).astype(np.int32)
+    return lay
+
+
+def layout_t2va(n_text, n_audio, grid, pad_to=256, drop_video_tail=0, name=None) -> Layout:
+    """Text, target audio, target video grid, then padding up to ``pad_to``.
+    Video and text rows use timestep index 0, audio rows index 1."""
+    t, h, w = grid
+    b = _Builder(name or f"t2va_{n_text}+{n_audio}+{t}x{h}x{w}")
+    b.add("text", TAG_TEXT, 0, text_positions(n_text))
+    b.add("audio", TAG_AUDIO, 1, audio_positions(n_audio))
+    vid = grid_positions(t, h, w)
+    if drop_video_tail:
+        vid = vid[: vid.shape[0] - drop_video_tail]
+    b.add("video", TAG_VIDEO, 0, vid)
+    n = b.n
+    npad = _round_up(n, pad_to) - n
+    if drop_video_tail:
+        npad = drop_video_tail
+    if npad:
+        b.add("pad", TAG_PAD, 0, pad_positions(npad))
+    return b.build()
+
+
+def layout_real_8k() -> Layout:
+    """8192 padless rows: 512 text, 256 audio, 7424 video on a (29, 16, 16) grid."""
+    return layout_t2va(512, 256, (29, 16, 16), name="real_8k")
+
+
+def layout_t2va_32k() -> Layout:
+    """32768 padless rows: 512 text, 1008 audio, 31248 video on (31, 24, 42):
+    124 frames at 1344x768 after 4x temporal and 32x spatial reduction."""
+    return layout_t2va(512, 1008, (31, 24, 42), name="t2va_32k")
+
+
+def layout_t2va_32k_padded() -> Layout:
+    """Variant of the 32k layout with 168 padding rows at the tail
+    (V = 32600, P = 168): the last 168 video rows are replaced by padding."""
+    return layout_t2va(512, 1008, (31, 24, 42), drop_video_tail=168, name="t2va_32k_pad168")
+
+
+def layout_ref2va() -> Layout:
+    """ref2va-shaped sequence: 512 text; 9 image references of 1x24x42 and
+    3 video references of 4x24x42 (conditioning tag, timestep index 2);
+    3 audio references of 128 rows (audio tag, index 2); 1008 target audio
+    rows (index 1); a 31x24x42 target video grid (index 0); then padding to a
+    multiple of 256. References advance one shared rotary time axis in order."""
+    b = _Builder("ref2va_54k")
+    b.add("text", TAG_TEXT, 0, text_positions(512))
+    clock = 0
+    for _ in range(9):
+        b.add("image_ref", TAG_COND, 2, grid_positions(1, 24, 42, t0=clock))
+        clock += 1
+    for _ in range(3):
+        b.add("video_ref", TAG_COND, 2, grid_positions(4, 24, 42, t0=clock))
+        clock += 4
+    for _ in range(3):
+        b.add("audio_ref", TAG_AUDIO, 2, audio_positions(128, t0=clock))
+        clock += 128
+    b.add("audio", TAG_AUDIO, 1, audio_positions(1008))
+    b.add("video", TAG_VIDEO, 0, grid_positions(31, 24, 42))
+    npad = _round_up(b.n, 256) - b.n
+    b.add("pad", TAG_PAD, 0, pad_positions(npad))
+    return b.build()
+
+
+def layout_two_time(base: Layout, seed=0) -> Layout:
+    """Two-time conditioning: timestep index = 2 * t_now + t_end, with
+    t_now, t_end drawn uniformly from {0, 1} per row (4 modulation sets)."""
+    rng = np.random.default_rng(seed + 2000)
+    t_now = rng.integers(0, 2, size=base.n)
+    t_end = rng.integers(0, 2, size=base.n)
+    return replace(base, name=base.name + "_twotime",
+                   tidx=(2 * t_now + t_end).astype(np.int32))
+
+
+# --------------------------------------------------------------------------
+# Named workloads
+# --------------------------------------------------------------------------
+
+WORKLOADS = {
+    "tiny_320": (TINY, layout_tiny),
+    "real_8k": (REAL, layout_real_8k),
+    "t2va_32k": (REAL, layout_t2va_32k),
+    "t2va_32k_pad168": (REAL, layout_t2va_32k_padded),
+    "ref2va_54k": (replace(REAL, n_t=3), layout_ref2va),
+    "w8a8_t2va_32k": (replace(REAL, n_t=4, quant=1), lambda: layout_two_time(layout_t2va_32k())),
+}
+
+
+def workload(name, seed=0):
+    dims, mk = WORKLOADS[name]
+    lay = mk(seed) if name == "tiny_320" else mk()
+    return dims, lay
+
+
+# --------------------------------------------------------------------------
+# Random tensors
+# --------------------------------------------------------------------------
+
+def _normal(rng, shape, std):
+    a = rng.standard_normal(size=shape, dtype=np.float32)
+    if std != 1.0:
+        a *= np.float32(std)
+    return a
+
+
+def to_bf16(a: np.ndarray) -> torch.Tensor:
+    """Round an fp32 array to bf16 (round to nearest even), as a CPU tensor."""
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16)
+
+
+@dataclass
+class Weights:
+    wqkv: torch.Tensor   # bf16 [3*H*D, C]: rows q heads, then k heads, then v heads
+    q_gain: torch.Tensor  # bf16 [D]
+    k_gain: torch.Tensor  # bf16 [D]
+    wo: torch.Tensor     # bf16 [C, H*D]
+    w13: torch.Tensor    # bf16 [2F, C]: rows 0..F-1 = W1 (gate), F..2F-1 = W3 (up)
+    w2: torch.Tensor     # bf16 [C, F]
+
+
+def make_weights(dims: Dims, seed=0, unit_gains=False) -> Weights:
+    rng = np.random.default_rng(seed + 10)
+    C, HD, F, D = dims.hidden, dims.hd, dims.ffn, dims.head_dim
+    wqkv = to_bf16(_normal(rng, (3 * HD, C), 1.0 / np.sqrt(C)))
+    wo = to_bf16(_normal(rng, (C, HD), 1.0 / np.sqrt(HD)))
+    w13 = to_bf16(_normal(rng, (2 * F, C), 1.0 / np.sqrt(C)))
+    w2 = to_bf16(_normal(rng, (C, F), 1.0 / np.sqrt(F)))
+    if unit_gains:
+        qg = torch.ones(D, dtype=torch.bfloat16)
+        kg = torch.ones(D, dtype=torch.bfloat16)
+    else:
+        qg = to_bf16(1.0 + _normal(rng, (D,), 0.1))
+        kg = to_bf16(1.0 + _normal(rng, (D,), 0.1))
+    return Weights(wqkv, qg, kg, wo, w13, w2)
+
+
+def make_x(dims: Dims, n: int, seed=0) -> torch.Tensor:
+    rng = np.random.default_rng(seed + 20)
+    return to_bf16(_normal(rng, (n, dims.hidden), 1.0))
+
+
+def make_table(dims: Dims, seed=0) -> torch.Tensor:
+    """fp32 [n_tags][n_t][6][C]; the 6 vectors are shift1, scale1, gate1,
+    shift2, scale2, gate2."""
+    rng = np.random.default_rng(seed + 30)
+    return torch.from_numpy(_normal(rng, (dims.n_tags, dims.n_t, 6, dims.hidden), 0.1))
+
+
+@dataclass
+class Inputs:
+    dims: Dims
+    layout: Layout
+    x: torch.Tensor       # bf16 [N, C]
+    table: torch.Tensor   # fp32 [n_tags, n_t, 6, C]
+    weights: Weights
+
+    @property
+    def tag(self):
+        return torch.from_numpy(self.layout.tag)
+
+    @property
+    def tidx(self):
+        return torch.from_numpy(self.layout.tidx)
+
+    @property
+    def pos(self):
+        return torch.from_numpy(self.layout.pos)
+
+
+def make_inputs(name_or_dims, layout: Layout | None = None, seed=0, unit_gains=False) -> Inputs:
+    if isinstance(name_or_dims, str):
+        dims, layout = workload(name_or_dims, seed)
+    else:
+        dims = name_or_dims
+    return Inputs(dims, layout, make_x(dims, layout.n, seed), make_table(dims, seed),
+                  make_weights(dims, seed, unit_gains))
+
+
+def sample_rows(layout: Layout, k=256, k_pad=8, seed=0) -> np.ndarray:
+    """Seeded subset of rows used to compare against the oracle on large
+    sequences: ``k`` non-padding rows plus up to ``k_pad`` padding rows."""
+    rng = np.random.default_rng(seed + 40)
+    valid = np.nonzero(layout.tag != TAG_PAD)[0]
+    pad = np.nonzero(layout.tag == TAG_PAD)[0]
+    rows = rng.choice(valid, size=min(k, valid.size), replace=False)
+    if pad.size:
+        rows = np.concatenate([rows, rng.choice(pad, size=min(k_pad, pad.size), replace=False)])
+    return np.sort(rows).astype(np.int64)

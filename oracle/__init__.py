@@ -1,0 +1,11 @@
+"""fp64 CPU oracle of one MiniMax-H3 transformer block (test infrastructure).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package; the CUDA library never does.
+"""
+from .h3_block import (  # noqa: F401
+    BlockOracle, adaln, apply_rope, attention, documents, int8_matmul_exact,
+    modulation, prepare_int8_weight, qk_rmsnorm, quantize_rows, rmsnorm,
+    rope_angles, rope_frequencies, rotate_blocks, silu, softmax, swiglu,
+    sylvester_hadamard, w8a8_linear,
+)
