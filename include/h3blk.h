@@ -1,0 +1,229 @@
+/*
+ * h3blk — forward of one MiniMax-H3 transformer block on a B200 (sm_100a).
+ *
+ * The block runs over ONE packed 1-D sequence of N rows (text, conditioning
+ * image/video, audio and target-video rows, plus optional padding rows) with
+ * full self-attention, per-row AdaLN modulation selected by a modality tag and
+ * a timestep index, per-head QK RMSNorm, 3D (t, h, w) rotary embedding and a
+ * SwiGLU feed-forward:
+ *
+ *   m      = table[tag[r]][tidx[r]]            (6 vectors; zeros for tag -1)
+ *   h1     = rmsnorm(x) * (1 + scale1) + shift1
+ *   q,k,v  = h1 Wqkv^T;  q = rope(rmsnorm_D(q) g_q),  k = rope(rmsnorm_D(k) g_k)
+ *   o      = softmax(q k^T / sqrt(D) + docmask) v      (doc(r) = tag[r] == -1)
+ *   x1     = x  + gate1 * (o Wo^T)
+ *   h2     = rmsnorm(x1) * (1 + scale2) + shift2
+ *   out    = x1 + gate2 * ((silu(h2 W1^T) * (h2 W3^T)) W2^T)
+ *
+ * Sources (page title, section):
+ *   "MiniMaxH3Transformer3DModel" (diffusers API page)
+ *     - introduction: one packed sequence, full self-attention, no
+ *       cross-attention, no per-modality block weights; the per-row modality
+ *       tag selects the AdaLN modulation; padding rows (tag -1) form their own
+ *       attention document;
+ *     - constructor: hidden_size, num_attention_heads x attention_head_dim
+ *       (larger than hidden), ffn_dim (SwiGLU), rope_theta, norm_eps of the
+ *       pre-attention / pre-feed-forward norms, qk_norm_eps of the per-head
+ *       query/key norms;
+ *     - forward: timestep_indices, token_tags, position_ids (seq_len, 3).
+ *   "HyperFlow H3 Flash Brings MiniMax H3 Video to One GPU",
+ *     "How it got smaller and faster": rotated W8A8 INT8 linears.
+ * The block's equations are not printed on the pages; the reading above
+ * (sequential AdaLN pre-norm block, gain-free RMSNorm pre-norms, modulation
+ * order shift/scale/gate x 2, adjacent-pair RoPE with per-axis frequencies
+ * theta^(-i/n)) is the one this library implements.
+ *
+ * Conventions for every entry point:
+ *   - Return value: H3BLK_OK (0) or one of the H3BLK_ERR_* codes below.
+ *     h3blk_error_string() gives a message. Nothing is thrown or aborted.
+ *   - Device pointers are CUDA global-memory pointers owned by the caller and
+ *     must be 16-byte aligned. The library never allocates device memory:
+ *     every intermediate lives in the caller's workspace.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream). Calls are asynchronous on it: no host synchronisation, except
+ *     in h3blk_check.
+ *   - Matrices are row-major; a linear's weight is [out_features, in_features].
+ */
+#ifndef H3BLK_H
+#define H3BLK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define H3BLK_API __attribute__((visibility("default")))
+#else
+#define H3BLK_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ------------------------------------------------------------------ status */
+#define H3BLK_OK 0
+#define H3BLK_ERR_INVALID_ARG 1 /* null / misaligned pointer, bad size, aliasing */
+#define H3BLK_ERR_UNSUPPORTED 2 /* a dimension this build does not handle */
+#define H3BLK_ERR_CUDA 3        /* a CUDA runtime / driver call failed */
+#define H3BLK_ERR_TIMEOUT 4     /* a kernel pipeline wait gave up (reported by h3blk_check) */
+#define H3BLK_ERR_BAD_INDEX 5   /* a tag / timestep index outside the table (h3blk_check) */
+
+/* ------------------------------------------------------------------ config */
+typedef struct {
+  int hidden;       /* C: channels of the residual stream (multiple of 128)          */
+  int heads;        /* H                                                               */
+  int head_dim;     /* D: 64 or 128                                                    */
+  int ffn;          /* F: SwiGLU inner dimension (multiple of 128)                     */
+  int n_tags;       /* modality tags 0..n_tags-1 (tag -1 = padding)                    */
+  int n_t;          /* distinct timestep indices 0..n_t-1                              */
+  int rope_pairs_t; /* rotary pairs driven by the t / h / w coordinate, in this order; */
+  int rope_pairs_h; /* their sum is <= head_dim/2 and the remaining pairs pass through */
+  int rope_pairs_w;
+  float rope_theta; /* frequency of pair i of an axis with n pairs: theta^(-i/n)       */
+  float norm_eps;   /* eps of the two AdaLN pre-norms                                  */
+  float qk_norm_eps;/* eps of the per-head q / k RMSNorm                               */
+  int quant;        /* 0: bf16 linears; 1: rotated W8A8 INT8 linears                   */
+} h3blk_config;
+
+typedef struct h3blk_ctx* h3blk_handle;
+
+/* Weights of one block (device pointers, caller-owned).
+ * quant == 0: all matrices bf16; s_* unused (may be NULL).
+ * quant == 1: matrices int8 as written by h3blk_prepare_int8_weights (input
+ *             channels rotated by the block-128 Hadamard transform), s_* the
+ *             fp32 per-output-channel scales. q_gain / k_gain stay bf16.
+ *   wqkv [3*H*D, C]  rows: q of heads 0..H-1, then k, then v
+ *   q_gain, k_gain [D]
+ *   wo   [C, H*D]
+ *   w13  [2F, C]     rows 0..F-1 = W1 (gate, through silu), F..2F-1 = W3 (up)
+ *   w2   [C, F]                                                              */
+typedef struct {
+  const void* wqkv;
+  const void* q_gain;
+  const void* k_gain;
+  const void* wo;
+  const void* w13;
+  const void* w2;
+  const float* s_qkv; /* [3*H*D] */
+  const float* s_o;   /* [C]     */
+  const float* s_13;  /* [2F]    */
+  const float* s_2;   /* [C]     */
+} h3blk_weights;
+
+/* Creates a handle from a configuration. Host-only: touches no GPU.
+ * INVALID_ARG for null pointers or non-positive sizes; UNSUPPORTED when
+ * hidden or ffn is not a multiple of 128, head_dim is not 64 or 128, heads *
+ * head_dim is not a multiple of 128, or the rotary pairs exceed head_dim/2.
+ * The handle owns only host memory; release it with h3blk_destroy. */
+H3BLK_API int h3blk_create(const h3blk_config* cfg, h3blk_handle* out);
+
+/* Releases a handle (NULL is ignored). */
+H3BLK_API void h3blk_destroy(h3blk_handle h);
+
+/* Workspace bytes h3blk_forward needs for n_rows rows (n_rows >= 1). */
+H3BLK_API int h3blk_workspace_bytes(h3blk_handle h, int64_t n_rows, size_t* bytes);
+
+/* Stage buffers inside the workspace, readable after h3blk_forward (for
+ * stage-by-stage checks). Layout of each stage, all row-major:
+ *   H3BLK_STAGE_H1, _H2        bf16 [N, C]      pre-norm outputs (bf16 path only)
+ *   H3BLK_STAGE_X1             bf16 [N, C]      residual after the attention branch
+ *   H3BLK_STAGE_QKV            bf16 [N, 3*H*D]  q | k | v after QK-norm + RoPE
+ *   H3BLK_STAGE_O              bf16 [N, H*D]    attention output
+ *   H3BLK_STAGE_A              bf16 [N, F]      SwiGLU output
+ *   H3BLK_STAGE_*_Q8           int8 [N, K]      rotated, quantised linear input (W8A8)
+ *   H3BLK_STAGE_*_SCALE        fp32 [N]         its per-row scale            (W8A8)
+ *   H3BLK_STAGE_ERROR          int32 [1]        device error bits of the last forward */
+enum {
+  H3BLK_STAGE_H1 = 0,
+  H3BLK_STAGE_QKV = 1,
+  H3BLK_STAGE_O = 2,
+  H3BLK_STAGE_X1 = 3,
+  H3BLK_STAGE_H2 = 4,
+  H3BLK_STAGE_A = 5,
+  H3BLK_STAGE_H1_Q8 = 6,
+  H3BLK_STAGE_H1_SCALE = 7,
+  H3BLK_STAGE_O_Q8 = 8,
+  H3BLK_STAGE_O_SCALE = 9,
+  H3BLK_STAGE_H2_Q8 = 10,
+  H3BLK_STAGE_H2_SCALE = 11,
+  H3BLK_STAGE_A_Q8 = 12,
+  H3BLK_STAGE_A_SCALE = 13,
+  H3BLK_STAGE_ERROR = 14,
+  H3BLK_STAGE_COUNT = 15
+};
+H3BLK_API int h3blk_stage_view(h3blk_handle h, int64_t n_rows, int stage, size_t* offset, size_t* bytes);
+
+/* One block forward over n_rows packed rows.
+ *   x         bf16 [N, C]            input rows
+ *   tag       int32 [N]              modality tag in [0, n_tags), -1 = padding
+ *   tidx      int32 [N]              timestep index in [0, n_t) (ignored for padding)
+ *   pos       int32 [N, 3]           (t, h, w) rotary coordinates
+ *   mod_table fp32 [n_tags][n_t][6][C]: shift1, scale1, gate1, shift2, scale2, gate2
+ *   w         weights (see h3blk_weights)
+ *   out       bf16 [N, C]            must not overlap x or the workspace
+ *   workspace >= h3blk_workspace_bytes(h, N) bytes of device memory
+ * Padding rows leave the block unchanged (out = x) and never influence other
+ * rows. Indices outside the table are not read: such rows get zero modulation
+ * and the error is reported by h3blk_check. */
+H3BLK_API int h3blk_forward(h3blk_handle h, int64_t n_rows, const void* x, const int32_t* tag, const int32_t* tidx,
+                  const int32_t* pos, const float* mod_table, const h3blk_weights* w, void* out,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream` and reads the device error word of the last forward
+ * that used `workspace`: *status = H3BLK_OK, H3BLK_ERR_BAD_INDEX or
+ * H3BLK_ERR_TIMEOUT. */
+H3BLK_API int h3blk_check(h3blk_handle h, int64_t n_rows, const void* workspace, void* stream, int* status);
+
+/* Per-kernel timing. When set, every later h3blk_forward on this handle
+ * records the caller's CUDA events (cudaEvent_t passed as void*) on its stream
+ * at H3BLK_TIMING_POINTS points: before each of the forward's kernel groups
+ * and after the last one. Interval i (events[i] -> events[i+1]) covers:
+ *   0 prep (error word reset + tile summary), 1 pre-attention norm (+ int8
+ *   quant), 2 QKV GEMM, 3 attention, 4 int8 quant of the attention output
+ *   (empty on the bf16 path), 5 out-projection GEMM, 6 pre-FFN norm, 7 FFN-up
+ *   GEMM + SwiGLU, 8 int8 quant of the SwiGLU output (empty on the bf16
+ *   path), 9 FFN-down GEMM.
+ * The events stay owned by the caller; n_events = 0 (or events = NULL)
+ * switches recording off. INVALID_ARG unless n_events is 0 or
+ * H3BLK_TIMING_POINTS. */
+#define H3BLK_TIMING_POINTS 11
+H3BLK_API int h3blk_set_kernel_events(h3blk_handle h, void* const* events, int n_events);
+
+/* --------------------------------------------------------------- W8A8 */
+/* Bytes of the int8 weight blob for this configuration. */
+H3BLK_API int h3blk_int8_weights_bytes(h3blk_handle h, size_t* bytes);
+
+/* Rotates (block-128 Hadamard on input channels, W' = W H / sqrt(128)) and
+ * quantises (per output channel, symmetric, s = amax/127) the bf16 weights in
+ * `bf16_in` into `blob` (>= h3blk_int8_weights_bytes). Fills *int8_out with
+ * pointers into the blob (q/k gains are copied there too). */
+H3BLK_API int h3blk_prepare_int8_weights(h3blk_handle h, const h3blk_weights* bf16_in, void* blob, size_t blob_bytes,
+                               h3blk_weights* int8_out, void* stream);
+
+/* ------------------------------------------------------- kernel-level calls */
+/* The block's building blocks, exposed for tests and for callers composing
+ * their own pipelines. All device pointers, all asynchronous on `stream`. */
+
+/* Block-128 Hadamard rotation of each row of a bf16 [rows, K] matrix (K a
+ * multiple of 128, <= 16384), then symmetric per-row int8 quantisation:
+ * q = clamp(rint(v / s), -127, 127), s = amax / 127 (s = 0, q = 0 for a zero row). */
+H3BLK_API int h3blk_rotate_quantize(int64_t rows, int K, const void* in_bf16, int8_t* out_q, float* out_scale, void* stream);
+
+/* Exact int8 GEMM: C[M, N] = A[M, K] B[N, K]^T with int32 accumulation and
+ * no rounding (K a multiple of 128, N a multiple of 128). */
+H3BLK_API int h3blk_gemm_s8_s32(int64_t M, int N, int K, const int8_t* A, const int8_t* B, int32_t* C, void* stream);
+
+/* bf16 GEMM: C[M, N] = A[M, K] B[N, K]^T, fp32 accumulation, bf16 output
+ * (K a multiple of 64, N a multiple of 128). */
+H3BLK_API int h3blk_gemm_bf16(int64_t M, int N, int K, const void* A, const void* B, void* C, void* stream);
+
+/* Message for a status code (static storage). */
+H3BLK_API const char* h3blk_error_string(int status);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+H3BLK_API int h3blk_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* H3BLK_H */

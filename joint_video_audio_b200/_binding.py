@@ -1,0 +1,182 @@
+"""ctypes binding of libh3blk (include/h3blk.h): the same entry points under
+the same names, plus argument marshalling for torch tensors. Every step of the
+block runs in the library's CUDA kernels; nothing here computes.
+
+If libh3blk.so is missing the import fails: there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libh3blk.so")
+
+H3BLK_OK = 0
+H3BLK_ERR_INVALID_ARG = 1
+H3BLK_ERR_UNSUPPORTED = 2
+H3BLK_ERR_CUDA = 3
+H3BLK_ERR_TIMEOUT = 4
+H3BLK_ERR_BAD_INDEX = 5
+
+STAGES = ["H1", "QKV", "O", "X1", "H2", "A", "H1_Q8", "H1_SCALE", "O_Q8", "O_SCALE",
+          "H2_Q8", "H2_SCALE", "A_Q8", "A_SCALE", "ERROR"]
+STAGE = {name: i for i, name in enumerate(STAGES)}
+
+# every symbol include/h3blk.h declares
+EXPORTS = ["h3blk_create", "h3blk_destroy", "h3blk_workspace_bytes", "h3blk_stage_view", "h3blk_forward",
+           "h3blk_check", "h3blk_int8_weights_bytes", "h3blk_prepare_int8_weights", "h3blk_rotate_quantize",
+           "h3blk_gemm_s8_s32", "h3blk_gemm_bf16", "h3blk_error_string", "h3blk_version",
+           "h3blk_set_kernel_events"]
+
+H3BLK_TIMING_POINTS = 11
+TIMING_INTERVALS = ["prep", "norm1", "qkv_gemm", "attention", "quant_o", "out_proj_gemm", "norm2",
+                    "ffn_up_gemm", "quant_a", "ffn_down_gemm"]
+
+
+class h3blk_config(C.Structure):
+    _fields_ = [("hidden", C.c_int), ("heads", C.c_int), ("head_dim", C.c_int), ("ffn", C.c_int),
+                ("n_tags", C.c_int), ("n_t", C.c_int), ("rope_pairs_t", C.c_int), ("rope_pairs_h", C.c_int),
+                ("rope_pairs_w", C.c_int), ("rope_theta", C.c_float), ("norm_eps", C.c_float),
+                ("qk_norm_eps", C.c_float), ("quant", C.c_int)]
+
+
+class h3blk_weights(C.Structure):
+    _fields_ = [("wqkv", C.c_void_p), ("q_gain", C.c_void_p), ("k_gain", C.c_void_p), ("wo", C.c_void_p),
+                ("w13", C.c_void_p), ("w2", C.c_void_p), ("s_qkv", C.c_void_p), ("s_o", C.c_void_p),
+                ("s_13", C.c_void_p), ("s_2", C.c_void_p)]
+
+
+class H3BlkError(RuntimeError):
+    def __init__(self, fn, status):
+        super().__init__(f"{fn} failed: status {status} ({error_string(status)})")
+        self.status = status
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing; build it with `python joint_video_audio_b200/build.py`")
+    lib = C.CDLL(LIB_PATH)
+    vp, i64, i32, sz = C.c_void_p, C.c_int64, C.c_int, C.c_size_t
+    sig = {
+        "h3blk_create": (i32, [C.POINTER(h3blk_config), C.POINTER(vp)]),
+        "h3blk_destroy": (None, [vp]),
+        "h3blk_workspace_bytes": (i32, [vp, i64, C.POINTER(sz)]),
+        "h3blk_stage_view": (i32, [vp, i64, i32, C.POINTER(sz), C.POINTER(sz)]),
+        "h3blk_forward": (i32, [vp, i64, vp, vp, vp, vp, vp, C.POINTER(h3blk_weights), vp, vp, sz, vp]),
+        "h3blk_check": (i32, [vp, i64, vp, vp, C.POINTER(i32)]),
+        "h3blk_int8_weights_bytes": (i32, [vp, C.POINTER(sz)]),
+        "h3blk_prepare_int8_weights": (i32, [vp, C.POINTER(h3blk_weights), vp, sz, C.POINTER(h3blk_weights), vp]),
+        "h3blk_rotate_quantize": (i32, [i64, i32, vp, vp, vp, vp]),
+        "h3blk_gemm_s8_s32": (i32, [i64, i32, i32, vp, vp, vp, vp]),
+        "h3blk_gemm_bf16": (i32, [i64, i32, i32, vp, vp, vp, vp]),
+        "h3blk_error_string": (C.c_char_p, [i32]),
+        "h3blk_version": (i32, []),
+        "h3blk_set_kernel_events": (i32, [vp, C.POINTER(vp), i32]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+def _check(fn, status):
+    if status != H3BLK_OK:
+        raise H3BlkError(fn, status)
+
+
+# ---------------------------------------------------------------- raw entry points
+
+def error_string(status: int) -> str:
+    return _lib.h3blk_error_string(status).decode()
+
+
+def h3blk_error_string(status: int) -> str:
+    return error_string(status)
+
+
+def h3blk_version() -> int:
+    return _lib.h3blk_version()
+
+
+def h3blk_create(cfg: h3blk_config) -> int:
+    h = C.c_void_p()
+    _check("h3blk_create", _lib.h3blk_create(C.byref(cfg), C.byref(h)))
+    return h.value
+
+
+def h3blk_create_status(cfg) -> int:
+    """Status code of h3blk_create (for argument-validation tests)."""
+    h = C.c_void_p()
+    st = _lib.h3blk_create(C.byref(cfg) if cfg is not None else None, C.byref(h))
+    if st == H3BLK_OK:
+        _lib.h3blk_destroy(h)
+    return st
+
+
+def h3blk_destroy(handle: int) -> None:
+    _lib.h3blk_destroy(handle)
+
+
+def h3blk_workspace_bytes(handle: int, n_rows: int) -> int:
+    n = C.c_size_t()
+    _check("h3blk_workspace_bytes", _lib.h3blk_workspace_bytes(handle, n_rows, C.byref(n)))
+    return n.value
+
+
+def h3blk_stage_view(handle: int, n_rows: int, stage) -> tuple[int, int]:
+    st = STAGE[stage] if isinstance(stage, str) else int(stage)
+    off, nb = C.c_size_t(), C.c_size_t()
+    _check("h3blk_stage_view", _lib.h3blk_stage_view(handle, n_rows, st, C.byref(off), C.byref(nb)))
+    return off.value, nb.value
+
+
+def h3blk_forward(handle, n_rows, x, tag, tidx, pos, mod_table, weights: h3blk_weights, out, workspace,
+                  workspace_bytes, stream) -> int:
+    """Raw call; pointers are ints. Returns the status code."""
+    return _lib.h3blk_forward(handle, n_rows, x, tag, tidx, pos, mod_table, C.byref(weights), out, workspace,
+                              workspace_bytes, stream)
+
+
+def h3blk_check(handle, n_rows, workspace, stream) -> int:
+    st = C.c_int()
+    _check("h3blk_check", _lib.h3blk_check(handle, n_rows, workspace, stream, C.byref(st)))
+    return st.value
+
+
+def h3blk_int8_weights_bytes(handle) -> int:
+    n = C.c_size_t()
+    _check("h3blk_int8_weights_bytes", _lib.h3blk_int8_weights_bytes(handle, C.byref(n)))
+    return n.value
+
+
+def h3blk_prepare_int8_weights(handle, bf16_in: h3blk_weights, blob, blob_bytes, stream) -> h3blk_weights:
+    out = h3blk_weights()
+    _check("h3blk_prepare_int8_weights",
+           _lib.h3blk_prepare_int8_weights(handle, C.byref(bf16_in), blob, blob_bytes, C.byref(out), stream))
+    return out
+
+
+def h3blk_rotate_quantize(rows, K, in_bf16, out_q, out_scale, stream) -> int:
+    return _lib.h3blk_rotate_quantize(rows, K, in_bf16, out_q, out_scale, stream)
+
+
+def h3blk_gemm_s8_s32(M, N, K, A, B, Cp, stream) -> int:
+    return _lib.h3blk_gemm_s8_s32(M, N, K, A, B, Cp, stream)
+
+
+def h3blk_gemm_bf16(M, N, K, A, B, Cp, stream) -> int:
+    return _lib.h3blk_gemm_bf16(M, N, K, A, B, Cp, stream)
+
+
+def h3blk_set_kernel_events(handle, events) -> None:
+    """events: sequence of H3BLK_TIMING_POINTS raw cudaEvent_t values (ints), or None."""
+    if not events:
+        _check("h3blk_set_kernel_events", _lib.h3blk_set_kernel_events(handle, None, 0))
+        return
+    arr = (C.c_void_p * len(events))(*events)
+    _check("h3blk_set_kernel_events", _lib.h3blk_set_kernel_events(handle, arr, len(events)))

@@ -1,0 +1,539 @@
+// C-ABI of libh3blk: argument validation, workspace layout and the launch
+// sequence of one MiniMax-H3 block forward (see include/h3blk.h).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <new>
+
+#include "../../include/h3blk.h"
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+using h3::GemmArgs;
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+
+// ------------------------------------------------------------------ device info
+struct DeviceInfo {
+  bool ready = false;
+  int num_sms = 0;
+};
+constexpr int kMaxDevices = 64;
+DeviceInfo g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::mutex g_mu;
+
+// Current device's SM count and the driver's tensor-map encoder.
+int device_info(int* num_sms, PFN_cuTensorMapEncodeTiled_v12000* encode) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return H3BLK_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+      return H3BLK_ERR_CUDA;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return H3BLK_ERR_CUDA;
+    if (major != 10 || minor != 0) return H3BLK_ERR_UNSUPPORTED;  // built for sm_100a only
+    d.num_sms = sms;
+    d.ready = true;
+  }
+  *num_sms = d.num_sms;
+  *encode = g_encode;
+  return H3BLK_OK;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? H3BLK_OK : H3BLK_ERR_CUDA; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+}  // namespace
+
+struct h3blk_ctx {
+  h3blk_config cfg;
+  h3::RopeTable rope;
+  cudaEvent_t events[H3BLK_TIMING_POINTS];
+  bool timing;
+};
+
+namespace {
+
+// Workspace layout: every stage buffer at a 256-byte aligned offset.
+struct Layout {
+  size_t off[H3BLK_STAGE_COUNT];
+  size_t len[H3BLK_STAGE_COUNT];
+  size_t tiles_off;
+  size_t total;
+};
+
+Layout make_layout(const h3blk_config& c, int64_t n) {
+  Layout L;
+  std::memset(&L, 0, sizeof(L));
+  const size_t N = (size_t)n, C = c.hidden, HD = (size_t)c.heads * c.head_dim, F = c.ffn;
+  size_t o = 0;
+  auto put = [&](int stage, size_t bytes) {
+    L.off[stage] = o;
+    L.len[stage] = bytes;
+    o = align256(o + bytes);
+  };
+  put(H3BLK_STAGE_ERROR, 4);
+  L.tiles_off = o;
+  o = align256(o + ((N + 127) / 128) * sizeof(h3::TileInfo));
+  const bool q = c.quant != 0;
+  if (!q) put(H3BLK_STAGE_H1, N * C * 2);
+  put(H3BLK_STAGE_QKV, N * 3 * HD * 2);
+  put(H3BLK_STAGE_O, N * HD * 2);
+  put(H3BLK_STAGE_X1, N * C * 2);
+  if (!q) put(H3BLK_STAGE_H2, N * C * 2);
+  put(H3BLK_STAGE_A, N * F * 2);
+  if (q) {
+    put(H3BLK_STAGE_H1_Q8, N * C);
+    put(H3BLK_STAGE_H1_SCALE, N * 4);
+    put(H3BLK_STAGE_O_Q8, N * HD);
+    put(H3BLK_STAGE_O_SCALE, N * 4);
+    put(H3BLK_STAGE_H2_Q8, N * C);
+    put(H3BLK_STAGE_H2_SCALE, N * 4);
+    put(H3BLK_STAGE_A_Q8, N * F);
+    put(H3BLK_STAGE_A_SCALE, N * 4);
+  }
+  L.total = o;
+  return L;
+}
+
+// Int8 weight blob layout.
+struct BlobLayout {
+  size_t wqkv, wo, w13, w2, s_qkv, s_o, s_13, s_2, q_gain, k_gain, total;
+};
+
+BlobLayout make_blob(const h3blk_config& c) {
+  const size_t C = c.hidden, HD = (size_t)c.heads * c.head_dim, F = c.ffn, D = c.head_dim;
+  BlobLayout b;
+  size_t o = 0;
+  auto put = [&](size_t bytes) {
+    const size_t at = o;
+    o = align256(o + bytes);
+    return at;
+  };
+  b.wqkv = put(3 * HD * C);
+  b.wo = put(C * HD);
+  b.w13 = put(2 * F * C);
+  b.w2 = put(C * F);
+  b.s_qkv = put(3 * HD * 4);
+  b.s_o = put(C * 4);
+  b.s_13 = put(2 * F * 4);
+  b.s_2 = put(C * 4);
+  b.q_gain = put(D * 2);
+  b.k_gain = put(D * 2);
+  b.total = o;
+  return b;
+}
+
+GemmArgs base_gemm(const h3blk_ctx* h, int* err) {
+  GemmArgs g;
+  std::memset(&g, 0, sizeof(g));
+  g.n_tags = h->cfg.n_tags;
+  g.n_t = h->cfg.n_t;
+  g.head_dim = h->cfg.head_dim;
+  g.hd = h->cfg.heads * h->cfg.head_dim;
+  g.qk_eps = h->cfg.qk_norm_eps;
+  g.rope = h->rope;
+  g.err = err;
+  g.int8 = h->cfg.quant != 0;
+  return g;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* h3blk_error_string(int status) {
+  switch (status) {
+    case H3BLK_OK: return "ok";
+    case H3BLK_ERR_INVALID_ARG: return "invalid argument (null or misaligned pointer, bad size, or aliasing)";
+    case H3BLK_ERR_UNSUPPORTED: return "unsupported dimension or device";
+    case H3BLK_ERR_CUDA: return "CUDA runtime or driver error";
+    case H3BLK_ERR_TIMEOUT: return "a kernel pipeline wait timed out";
+    case H3BLK_ERR_BAD_INDEX: return "a modality tag or timestep index lies outside the modulation table";
+    default: return "unknown status";
+  }
+}
+
+int h3blk_version(void) { return kVersion; }
+
+int h3blk_create(const h3blk_config* cfg, h3blk_handle* out) {
+  if (!cfg || !out) return H3BLK_ERR_INVALID_ARG;
+  *out = nullptr;
+  const h3blk_config& c = *cfg;
+  if (c.hidden <= 0 || c.heads <= 0 || c.head_dim <= 0 || c.ffn <= 0 || c.n_tags <= 0 || c.n_t <= 0 ||
+      c.rope_pairs_t < 0 || c.rope_pairs_h < 0 || c.rope_pairs_w < 0 || !(c.rope_theta > 0.f) ||
+      !(c.norm_eps >= 0.f) || !(c.qk_norm_eps >= 0.f) || (c.quant != 0 && c.quant != 1))
+    return H3BLK_ERR_INVALID_ARG;
+  if (c.hidden % 128 || c.ffn % 128 || (c.head_dim != 64 && c.head_dim != 128) || (c.heads * c.head_dim) % 128 ||
+      c.rope_pairs_t + c.rope_pairs_h + c.rope_pairs_w > c.head_dim / 2 || c.hidden > 6144 || c.ffn > 16384 ||
+      c.heads * c.head_dim > 16384)
+    return H3BLK_ERR_UNSUPPORTED;
+  h3blk_ctx* h = new (std::nothrow) h3blk_ctx;
+  if (!h) return H3BLK_ERR_INVALID_ARG;
+  h->cfg = c;
+  h->timing = false;
+  for (auto& e : h->events) e = nullptr;
+  const int pairs[3] = {c.rope_pairs_t, c.rope_pairs_h, c.rope_pairs_w};
+  int j = 0;
+  for (int axis = 0; axis < 3; ++axis)
+    for (int i = 0; i < pairs[axis]; ++i, ++j) {
+      h->rope.axis[j] = (int8_t)axis;
+      h->rope.freq[j] = (float)std::pow((double)c.rope_theta, -(double)i / (double)pairs[axis]);
+    }
+  for (; j < h3::kMaxRopePairs; ++j) {
+    h->rope.axis[j] = 3;
+    h->rope.freq[j] = 0.f;
+  }
+  *out = h;
+  return H3BLK_OK;
+}
+
+void h3blk_destroy(h3blk_handle h) { delete h; }
+
+int h3blk_set_kernel_events(h3blk_handle h, void* const* events, int n_events) {
+  if (!h) return H3BLK_ERR_INVALID_ARG;
+  if (n_events == 0 || !events) {
+    h->timing = false;
+    return H3BLK_OK;
+  }
+  if (n_events != H3BLK_TIMING_POINTS) return H3BLK_ERR_INVALID_ARG;
+  for (int i = 0; i < n_events; ++i) {
+    if (!events[i]) return H3BLK_ERR_INVALID_ARG;
+    h->events[i] = reinterpret_cast<cudaEvent_t>(events[i]);
+  }
+  h->timing = true;
+  return H3BLK_OK;
+}
+
+int h3blk_workspace_bytes(h3blk_handle h, int64_t n_rows, size_t* bytes) {
+  if (!h || !bytes || n_rows < 1) return H3BLK_ERR_INVALID_ARG;
+  *bytes = make_layout(h->cfg, n_rows).total;
+  return H3BLK_OK;
+}
+
+int h3blk_stage_view(h3blk_handle h, int64_t n_rows, int stage, size_t* offset, size_t* bytes) {
+  if (!h || !offset || !bytes || n_rows < 1 || stage < 0 || stage >= H3BLK_STAGE_COUNT) return H3BLK_ERR_INVALID_ARG;
+  const Layout L = make_layout(h->cfg, n_rows);
+  if (L.len[stage] == 0) return H3BLK_ERR_UNSUPPORTED;  // stage not produced in this mode
+  *offset = L.off[stage];
+  *bytes = L.len[stage];
+  return H3BLK_OK;
+}
+
+int h3blk_forward(h3blk_handle h, int64_t n_rows, const void* x, const int32_t* tag, const int32_t* tidx,
+                  const int32_t* pos, const float* mod_table, const h3blk_weights* w, void* out, void* workspace,
+                  size_t workspace_bytes, void* stream) {
+  if (!h || !w || n_rows < 1 || !x || !tag || !tidx || !pos || !mod_table || !out || !workspace)
+    return H3BLK_ERR_INVALID_ARG;
+  const h3blk_config& c = h->cfg;
+  const bool q = c.quant != 0;
+  if (!w->wqkv || !w->q_gain || !w->k_gain || !w->wo || !w->w13 || !w->w2) return H3BLK_ERR_INVALID_ARG;
+  if (q && (!w->s_qkv || !w->s_o || !w->s_13 || !w->s_2)) return H3BLK_ERR_INVALID_ARG;
+  const void* ptrs[] = {x, tag, tidx, pos, mod_table, out, workspace, w->wqkv, w->wo, w->w13, w->w2};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return H3BLK_ERR_INVALID_ARG;
+  const Layout L = make_layout(c, n_rows);
+  if (workspace_bytes < L.total) return H3BLK_ERR_INVALID_ARG;
+  const size_t N = (size_t)n_rows, C = c.hidden, HD = (size_t)c.heads * c.head_dim, F = c.ffn;
+  if (overlap(out, N * C * 2, x, N * C * 2) || overlap(out, N * C * 2, workspace, L.total) ||
+      overlap(x, N * C * 2, workspace, L.total))
+    return H3BLK_ERR_INVALID_ARG;
+  int sms = 0;
+  PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+  int st = device_info(&sms, &enc);
+  if (st != H3BLK_OK) return st;
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  auto buf = [&](int stage) { return ws + L.off[stage]; };
+  int* err = reinterpret_cast<int*>(buf(H3BLK_STAGE_ERROR));
+  h3::TileInfo* tiles = reinterpret_cast<h3::TileInfo*>(ws + L.tiles_off);
+  auto* xb = static_cast<const __nv_bfloat16*>(x);
+  auto* qkv = reinterpret_cast<__nv_bfloat16*>(buf(H3BLK_STAGE_QKV));
+  auto* o = reinterpret_cast<__nv_bfloat16*>(buf(H3BLK_STAGE_O));
+  auto* x1 = reinterpret_cast<__nv_bfloat16*>(buf(H3BLK_STAGE_X1));
+  auto* a = reinterpret_cast<__nv_bfloat16*>(buf(H3BLK_STAGE_A));
+
+#define H3_TRY(expr)                       \
+  do {                                     \
+    cudaError_t e_ = (expr);               \
+    if (e_ != cudaSuccess) return H3BLK_ERR_CUDA; \
+  } while (0)
+
+  auto mark = [&](int i) -> cudaError_t { return h->timing ? cudaEventRecord(h->events[i], s) : cudaSuccess; };
+  H3_TRY(mark(0));
+  H3_TRY(cudaMemsetAsync(err, 0, sizeof(int), s));
+  H3_TRY(h3::launch_tile_info(tag, tidx, n_rows, c.n_tags, c.n_t, tiles, err, s));
+
+  // ---- pre-attention AdaLN + RMSNorm
+  h3::ModNormArgs mn;
+  std::memset(&mn, 0, sizeof(mn));
+  mn.x = xb;
+  mn.tag = tag;
+  mn.tidx = tidx;
+  mn.table = mod_table;
+  mn.n = n_rows;
+  mn.C = c.hidden;
+  mn.n_tags = c.n_tags;
+  mn.n_t = c.n_t;
+  mn.shift_idx = 0;
+  mn.scale_idx = 1;
+  mn.eps = c.norm_eps;
+  if (q) {
+    mn.out_q = reinterpret_cast<int8_t*>(buf(H3BLK_STAGE_H1_Q8));
+    mn.out_scale = reinterpret_cast<float*>(buf(H3BLK_STAGE_H1_SCALE));
+  } else {
+    mn.out_bf16 = reinterpret_cast<__nv_bfloat16*>(buf(H3BLK_STAGE_H1));
+  }
+  H3_TRY(mark(1));
+  H3_TRY(h3::launch_modnorm(mn, s));
+
+  // ---- QKV projection + QK-RMSNorm + RoPE
+  GemmArgs g = base_gemm(h, err);
+  g.A = q ? (const void*)buf(H3BLK_STAGE_H1_Q8) : (const void*)buf(H3BLK_STAGE_H1);
+  g.B = w->wqkv;
+  g.M = n_rows;
+  g.N = (int)(3 * HD);
+  g.Nb = (int)(3 * HD);
+  g.K = c.hidden;
+  g.epi = h3::kEpiQKV;
+  g.out = qkv;
+  g.ld_out = 3 * HD;
+  g.q_gain = static_cast<const __nv_bfloat16*>(w->q_gain);
+  g.k_gain = static_cast<const __nv_bfloat16*>(w->k_gain);
+  g.pos = pos;
+  g.s_a = q ? reinterpret_cast<const float*>(buf(H3BLK_STAGE_H1_SCALE)) : nullptr;
+  g.s_b = w->s_qkv;
+  H3_TRY(mark(2));
+  H3_TRY(h3::launch_gemm(g, enc, sms, s));
+
+  // ---- attention
+  h3::AttnArgs at;
+  at.qkv = qkv;
+  at.o = o;
+  at.tag = tag;
+  at.tiles = tiles;
+  at.n = n_rows;
+  at.heads = c.heads;
+  at.head_dim = c.head_dim;
+  at.err = err;
+  H3_TRY(mark(3));
+  H3_TRY(h3::launch_attention(at, enc, s));
+  H3_TRY(mark(4));
+
+  // ---- out-projection + gated residual
+  if (q)
+    H3_TRY(h3::launch_rotate_quant(o, n_rows, (int)HD, reinterpret_cast<int8_t*>(buf(H3BLK_STAGE_O_Q8)),
+                                   reinterpret_cast<float*>(buf(H3BLK_STAGE_O_SCALE)), s));
+  g = base_gemm(h, err);
+  g.A = q ? (const void*)buf(H3BLK_STAGE_O_Q8) : (const void*)o;
+  g.B = w->wo;
+  g.M = n_rows;
+  g.N = c.hidden;
+  g.Nb = c.hidden;
+  g.K = (int)HD;
+  g.epi = h3::kEpiResid;
+  g.out = x1;
+  g.ld_out = C;
+  g.resid = xb;
+  g.table = mod_table;
+  g.tag = tag;
+  g.tidx = tidx;
+  g.gate_idx = 2;
+  g.s_a = q ? reinterpret_cast<const float*>(buf(H3BLK_STAGE_O_SCALE)) : nullptr;
+  g.s_b = w->s_o;
+  H3_TRY(mark(5));
+  H3_TRY(h3::launch_gemm(g, enc, sms, s));
+  H3_TRY(mark(6));
+
+  // ---- pre-FFN AdaLN + RMSNorm
+  mn.x = x1;
+  mn.shift_idx = 3;
+  mn.scale_idx = 4;
+  if (q) {
+    mn.out_q = reinterpret_cast<int8_t*>(buf(H3BLK_STAGE_H2_Q8));
+    mn.out_scale = reinterpret_cast<float*>(buf(H3BLK_STAGE_H2_SCALE));
+  } else {
+    mn.out_bf16 = reinterpret_cast<__nv_bfloat16*>(buf(H3BLK_STAGE_H2));
+  }
+  H3_TRY(h3::launch_modnorm(mn, s));
+
+  // ---- FFN up (W1 | W3) + SwiGLU
+  g = base_gemm(h, err);
+  g.A = q ? (const void*)buf(H3BLK_STAGE_H2_Q8) : (const void*)buf(H3BLK_STAGE_H2);
+  g.B = w->w13;
+  g.M = n_rows;
+  g.N = c.ffn;
+  g.Nb = 2 * c.ffn;
+  g.K = c.hidden;
+  g.epi = h3::kEpiSwiGLU;
+  g.out = a;
+  g.ld_out = F;
+  g.s_a = q ? reinterpret_cast<const float*>(buf(H3BLK_STAGE_H2_SCALE)) : nullptr;
+  g.s_b = w->s_13;
+  H3_TRY(mark(7));
+  H3_TRY(h3::launch_gemm(g, enc, sms, s));
+  H3_TRY(mark(8));
+
+  // ---- FFN down + gated residual
+  if (q)
+    H3_TRY(h3::launch_rotate_quant(a, n_rows, (int)F, reinterpret_cast<int8_t*>(buf(H3BLK_STAGE_A_Q8)),
+                                   reinterpret_cast<float*>(buf(H3BLK_STAGE_A_SCALE)), s));
+  g = base_gemm(h, err);
+  g.A = q ? (const void*)buf(H3BLK_STAGE_A_Q8) : (const void*)a;
+  g.B = w->w2;
+  g.M = n_rows;
+  g.N = c.hidden;
+  g.Nb = c.hidden;
+  g.K = c.ffn;
+  g.epi = h3::kEpiResid;
+  g.out = out;
+  g.ld_out = C;
+  g.resid = x1;
+  g.table = mod_table;
+  g.tag = tag;
+  g.tidx = tidx;
+  g.gate_idx = 5;
+  g.s_a = q ? reinterpret_cast<const float*>(buf(H3BLK_STAGE_A_SCALE)) : nullptr;
+  g.s_b = w->s_2;
+  H3_TRY(mark(9));
+  H3_TRY(h3::launch_gemm(g, enc, sms, s));
+  H3_TRY(mark(10));
+  return H3BLK_OK;
+}
+
+int h3blk_check(h3blk_handle h, int64_t n_rows, const void* workspace, void* stream, int* status) {
+  if (!h || !workspace || !status || n_rows < 1) return H3BLK_ERR_INVALID_ARG;
+  const Layout L = make_layout(h->cfg, n_rows);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return H3BLK_ERR_CUDA;
+  int bits = 0;
+  if (cudaMemcpy(&bits, static_cast<const uint8_t*>(workspace) + L.off[H3BLK_STAGE_ERROR], sizeof(int),
+                 cudaMemcpyDeviceToHost) != cudaSuccess)
+    return H3BLK_ERR_CUDA;
+  if (bits & (h3::kErrTimeoutGemm | h3::kErrTimeoutAttn))
+    *status = H3BLK_ERR_TIMEOUT;
+  else if (bits & h3::kErrBadIndex)
+    *status = H3BLK_ERR_BAD_INDEX;
+  else
+    *status = H3BLK_OK;
+  return H3BLK_OK;
+}
+
+int h3blk_int8_weights_bytes(h3blk_handle h, size_t* bytes) {
+  if (!h || !bytes) return H3BLK_ERR_INVALID_ARG;
+  *bytes = make_blob(h->cfg).total;
+  return H3BLK_OK;
+}
+
+int h3blk_prepare_int8_weights(h3blk_handle h, const h3blk_weights* in, void* blob, size_t blob_bytes,
+                               h3blk_weights* out, void* stream) {
+  if (!h || !in || !blob || !out) return H3BLK_ERR_INVALID_ARG;
+  if (!in->wqkv || !in->q_gain || !in->k_gain || !in->wo || !in->w13 || !in->w2) return H3BLK_ERR_INVALID_ARG;
+  const h3blk_config& c = h->cfg;
+  const BlobLayout b = make_blob(c);
+  if (blob_bytes < b.total || !aligned16(blob)) return H3BLK_ERR_INVALID_ARG;
+  const void* ptrs[] = {in->wqkv, in->wo, in->w13, in->w2};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return H3BLK_ERR_INVALID_ARG;
+  int sms = 0;
+  PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+  int st = device_info(&sms, &enc);
+  if (st != H3BLK_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* bl = static_cast<uint8_t*>(blob);
+  const int64_t C = c.hidden, HD = (int64_t)c.heads * c.head_dim, F = c.ffn;
+  auto rq = [&](const void* w, int64_t rows, int K, size_t qo, size_t so) {
+    return h3::launch_rotate_quant(static_cast<const __nv_bfloat16*>(w), rows, K,
+                                   reinterpret_cast<int8_t*>(bl + qo), reinterpret_cast<float*>(bl + so), s);
+  };
+  if (rq(in->wqkv, 3 * HD, (int)C, b.wqkv, b.s_qkv) != cudaSuccess) return H3BLK_ERR_CUDA;
+  if (rq(in->wo, C, (int)HD, b.wo, b.s_o) != cudaSuccess) return H3BLK_ERR_CUDA;
+  if (rq(in->w13, 2 * F, (int)C, b.w13, b.s_13) != cudaSuccess) return H3BLK_ERR_CUDA;
+  if (rq(in->w2, C, (int)F, b.w2, b.s_2) != cudaSuccess) return H3BLK_ERR_CUDA;
+  if (cudaMemcpyAsync(bl + b.q_gain, in->q_gain, c.head_dim * 2, cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(bl + b.k_gain, in->k_gain, c.head_dim * 2, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return H3BLK_ERR_CUDA;
+  out->wqkv = bl + b.wqkv;
+  out->wo = bl + b.wo;
+  out->w13 = bl + b.w13;
+  out->w2 = bl + b.w2;
+  out->s_qkv = reinterpret_cast<const float*>(bl + b.s_qkv);
+  out->s_o = reinterpret_cast<const float*>(bl + b.s_o);
+  out->s_13 = reinterpret_cast<const float*>(bl + b.s_13);
+  out->s_2 = reinterpret_cast<const float*>(bl + b.s_2);
+  out->q_gain = bl + b.q_gain;
+  out->k_gain = bl + b.k_gain;
+  return H3BLK_OK;
+}
+
+int h3blk_rotate_quantize(int64_t rows, int K, const void* in_bf16, int8_t* out_q, float* out_scale, void* stream) {
+  if (rows < 0 || K <= 0 || K % 128 || K > 16384 || !in_bf16 || !out_q || !out_scale) return H3BLK_ERR_INVALID_ARG;
+  if (!aligned16(in_bf16) || !aligned16(out_q) || !aligned16(out_scale)) return H3BLK_ERR_INVALID_ARG;
+  int sms = 0;
+  PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+  int st = device_info(&sms, &enc);
+  if (st != H3BLK_OK) return st;
+  return cuda_status(h3::launch_rotate_quant(static_cast<const __nv_bfloat16*>(in_bf16), rows, K, out_q, out_scale,
+                                             reinterpret_cast<cudaStream_t>(stream)));
+}
+
+static int plain_gemm(int64_t M, int N, int K, const void* A, const void* B, void* C, void* stream, bool int8) {
+  if (M < 0 || N <= 0 || K <= 0 || !A || !B || !C) return H3BLK_ERR_INVALID_ARG;
+  if (N % 128 || K % (int8 ? 128 : 64)) return H3BLK_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(C)) return H3BLK_ERR_INVALID_ARG;
+  int sms = 0;
+  PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+  int st = device_info(&sms, &enc);
+  if (st != H3BLK_OK) return st;
+  GemmArgs g;
+  std::memset(&g, 0, sizeof(g));
+  g.A = A;
+  g.B = B;
+  g.M = M;
+  g.N = N;
+  g.Nb = N;
+  g.K = K;
+  g.int8 = int8;
+  g.epi = int8 ? h3::kEpiStoreS32 : h3::kEpiStoreBf16;
+  g.out = C;
+  g.ld_out = N;
+  g.err = nullptr;  // a standalone GEMM that times out just stops; C is then incomplete
+  return cuda_status(h3::launch_gemm(g, enc, sms, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int h3blk_gemm_s8_s32(int64_t M, int N, int K, const int8_t* A, const int8_t* B, int32_t* C, void* stream) {
+  return plain_gemm(M, N, K, A, B, C, stream, true);
+}
+
+int h3blk_gemm_bf16(int64_t M, int N, int K, const void* A, const void* B, void* C, void* stream) {
+  return plain_gemm(M, N, K, A, B, C, stream, false);
+}
+
+}  // extern "C"

@@ -1,0 +1,468 @@
+// Persistent, warp-specialised tcgen05 GEMM  C[M, N] = A[M, K] * B[N, K]^T
+// with the block's fused epilogues (K2a/K2b/K2c/K2d, and the int8 K5).
+//
+//   warp 0      TMA producer: A tile 128 x 128 B and B tile 256 x 128 B per stage
+//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
+//   warps 2..5  epilogue: tcgen05.ld of the fp32 / s32 accumulator (thread =
+//               output row), fused math, 16-byte global stores
+//
+// Accumulators are double-buffered in tensor memory (2 x 256 columns) so the
+// epilogue of tile i overlaps the main loop of tile i+1. Operands are staged by
+// TMA with the 128-byte swizzle the UMMA descriptors expect.
+//
+// Fused epilogues (sources: "MiniMaxH3Transformer3DModel", diffusers API
+// page, constructor: qk_norm_eps of the per-head query/key norms, rope_theta;
+// introduction: AdaLN modulation per modality tag; ffn_dim of the SwiGLU):
+//   kEpiQKV    q, k: per-head RMSNorm (fp32) * gain, then 3D RoPE on adjacent
+//              pairs; v: stored as is. Output [M, 3*H*D] bf16.
+//   kEpiResid  out = resid + gate[tag][tidx] * acc (padding rows: out = resid).
+//   kEpiSwiGLU B holds W1 rows then W3 rows; tile j loads W1 rows j*128.. and W3
+//              rows j*128.. into its two 128-column halves: out = silu(g) * u.
+//   kEpiStoreS32  raw int32 accumulators (exactness tests of the int8 path).
+// int8 mode ("HyperFlow H3 Flash ...", "How it got smaller and faster":
+// rotated W8A8): kind::i8, s32 accumulators, value = acc * s_a[row] * s_b[col].
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace h3 {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int kRowBytes = 128;  // one K-block per stage: 64 bf16 or 128 int8
+constexpr int kStages = 4;
+constexpr int kAStage = BM * kRowBytes;  // 16 KB
+constexpr int kBStage = BN * kRowBytes;  // 32 KB
+constexpr int kThreads = 192;
+constexpr int kTmemCols = 512;  // two 256-column fp32 accumulators
+constexpr int kGroupN = 8;      // tile raster: 8 N-tiles share each pass over M
+constexpr size_t kSmemBytes = 1024 + (size_t)kStages * (kAStage + kBStage) + 256;
+
+struct Smem {
+  uint8_t* a;
+  uint8_t* b;
+  uint64_t* full;
+  uint64_t* empty;
+  uint64_t* tfull;
+  uint64_t* tempty;
+  uint64_t* drain;
+  uint32_t* tmem_base;
+  int* abort;
+};
+
+__device__ __forceinline__ Smem carve(uint8_t* raw) {
+  const uint32_t base = smem_u32(raw);
+  const uint32_t pad = ((base + 1023u) & ~1023u) - base;
+  uint8_t* p = raw + pad;
+  Smem s;
+  s.a = p;
+  s.b = p + kStages * kAStage;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(p + kStages * (kAStage + kBStage));
+  s.full = bars;
+  s.empty = bars + kStages;
+  s.tfull = bars + 2 * kStages;
+  s.tempty = bars + 2 * kStages + 2;
+  s.drain = bars + 2 * kStages + 4;
+  s.tmem_base = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 5);
+  s.abort = reinterpret_cast<int*>(bars + 2 * kStages + 6);
+  return s;
+}
+
+struct TileCoord {
+  int m, n;
+};
+
+__device__ __forceinline__ TileCoord tile_coord(int t, int tiles_m, int tiles_n) {
+  const int group = t / (kGroupN * tiles_m);
+  const int first_n = group * kGroupN;
+  const int gn = min(kGroupN, tiles_n - first_n);
+  const int idx = t - group * kGroupN * tiles_m;
+  return {idx / gn, first_n + idx % gn};
+}
+
+__device__ __forceinline__ void fail(const Smem& s, int* err) {
+  if (err) atomicOr(err, kErrTimeoutGemm);
+  *reinterpret_cast<volatile int*>(s.abort) = 1;
+}
+
+// fp32 value of accumulator register j of a chunk starting at column `col`
+template <bool INT8>
+__device__ __forceinline__ float acc_value(uint32_t r, float sa, const float* sb, int col) {
+  if (INT8) return (float)(int)r * sa * __ldg(sb + col);
+  return __uint_as_float(r);
+}
+
+__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&v)[32]) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint4 o;
+    o.x = pack_bf16x2(v[8 * i + 0], v[8 * i + 1]);
+    o.y = pack_bf16x2(v[8 * i + 2], v[8 * i + 3]);
+    o.z = pack_bf16x2(v[8 * i + 4], v[8 * i + 5]);
+    o.w = pack_bf16x2(v[8 * i + 6], v[8 * i + 7]);
+    d[i] = o;
+  }
+}
+
+template <bool INT8>
+__device__ __forceinline__ void load_chunk(uint32_t taddr, float sa, const float* sb, int col, float (&v)[32]) {
+  uint32_t r[32];
+  tmem_ld32(taddr, r);
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = acc_value<INT8>(r[j], sa, sb, col + j);
+}
+
+// ------------------------------------------------------------------ epilogue
+template <int EPI, bool INT8>
+__device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tacc, int64_t row, bool row_ok, int n_tile) {
+  const float sa = (INT8 && row_ok) ? __ldg(p.s_a + row) : 0.f;
+  if (EPI == kEpiSwiGLU) {
+    const int col0 = n_tile * 128;
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      float g[32], u[32];
+      load_chunk<INT8>(tacc + c * 32, sa, p.s_b, col0 + c * 32, g);
+      load_chunk<INT8>(tacc + 128 + c * 32, sa, p.s_b, p.N + col0 + c * 32, u);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) g[j] = g[j] / (1.f + __expf(-g[j])) * u[j];
+      if (row_ok) store_bf16x32(reinterpret_cast<__nv_bfloat16*>(p.out) + row * p.ld_out + col0 + c * 32, g);
+    }
+    return;
+  }
+  const int n0 = n_tile * BN;
+  if (EPI == kEpiStoreS32) {
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      if (n0 + c * 32 >= p.N) break;
+      uint32_t r[32];
+      tmem_ld32(tacc + c * 32, r);
+      if (row_ok) {
+        uint4* d = reinterpret_cast<uint4*>(reinterpret_cast<int32_t*>(p.out) + row * p.ld_out + n0 + c * 32);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) d[i] = make_uint4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
+      }
+    }
+    return;
+  }
+  if (EPI == kEpiStoreBf16 || EPI == kEpiResid) {
+    const float* gate = nullptr;
+    if (EPI == kEpiResid && row_ok) {
+      const int tg = p.tag[row], ti = p.tidx[row];
+      if (tg >= 0 && tg < p.n_tags && ti >= 0 && ti < p.n_t)
+        gate = p.table + (((int64_t)tg * p.n_t + ti) * 6 + p.gate_idx) * p.N;
+    }
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      const int col = n0 + c * 32;
+      if (col >= p.N) break;
+      float v[32];
+      load_chunk<INT8>(tacc + c * 32, sa, p.s_b, col, v);
+      if (!row_ok) continue;
+      __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + row * p.ld_out + col;
+      if (EPI == kEpiResid) {
+        const uint4* rs = reinterpret_cast<const uint4*>(p.resid + row * (int64_t)p.N + col);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint4 q = __ldg(rs + i);
+          const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const float2 x2 = unpack_bf16x2(w[h]);
+            const int j = 8 * i + 2 * h;
+            if (gate) {
+              const float2 g2 = __ldg(reinterpret_cast<const float2*>(gate + col + j));
+              v[j] = fmaf(g2.x, v[j], x2.x);
+              v[j + 1] = fmaf(g2.y, v[j + 1], x2.y);
+            } else {
+              v[j] = x2.x;
+              v[j + 1] = x2.y;
+            }
+          }
+        }
+      }
+      store_bf16x32(dst, v);
+    }
+    return;
+  }
+  if (EPI == kEpiQKV) {
+    const int D = p.head_dim;
+    int pos3[3] = {0, 0, 0};
+    if (row_ok) {
+      pos3[0] = __ldg(p.pos + row * 3 + 0);
+      pos3[1] = __ldg(p.pos + row * 3 + 1);
+      pos3[2] = __ldg(p.pos + row * 3 + 2);
+    }
+#pragma unroll 1
+    for (int hh = 0; hh < BN / D; ++hh) {
+      const int col0 = n0 + hh * D;
+      if (col0 >= p.N) break;
+      const int region = col0 / p.hd;  // 0 q, 1 k, 2 v
+      const uint32_t th = tacc + hh * D;
+      __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + row * p.ld_out + col0;
+      if (region == 2) {
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          float v[32];
+          load_chunk<INT8>(th + c * 32, sa, p.s_b, col0 + c * 32, v);
+          if (row_ok) store_bf16x32(dst + c * 32, v);
+        }
+        continue;
+      }
+      float ss = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        float v[32];
+        load_chunk<INT8>(th + c * 32, sa, p.s_b, col0 + c * 32, v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) ss = fmaf(v[j], v[j], ss);
+      }
+      const float rstd = rsqrtf(ss / (float)D + p.qk_eps);
+      const __nv_bfloat16* gain = region == 0 ? p.q_gain : p.k_gain;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        float v[32];
+        load_chunk<INT8>(th + c * 32, sa, p.s_b, col0 + c * 32, v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = v[j] * rstd * __bfloat162float(gain[c * 32 + j]);
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          const int pair = c * 16 + q;
+          const int ax = p.rope.axis[pair];
+          if (ax < 3) {
+            float sn, cs;
+            const int pv = ax == 0 ? pos3[0] : (ax == 1 ? pos3[1] : pos3[2]);
+            sincosf((float)pv * p.rope.freq[pair], &sn, &cs);
+            const float a = v[2 * q], b = v[2 * q + 1];
+            v[2 * q] = a * cs - b * sn;
+            v[2 * q + 1] = a * sn + b * cs;
+          }
+        }
+        if (row_ok) store_bf16x32(dst + c * 32, v);
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ kernel
+template <int EPI, bool INT8>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const GemmArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  const Smem s = carve(smem_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tiles_m = (int)((p.M + BM - 1) / BM);
+  const int tiles_n = EPI == kEpiSwiGLU ? p.N / 128 : (p.N + BN - 1) / BN;
+  const int num_tiles = tiles_m * tiles_n;
+  const int num_kb = p.K / (INT8 ? 128 : 64);
+  volatile int* abort = s.abort;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.tfull[i], 1);
+      mbar_init(&s.tempty[i], 4);  // one arrival per epilogue warp
+    }
+    mbar_init(s.drain, 1);
+    *s.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(s.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *s.tmem_base;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      long issued = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        const TileCoord tc = tile_coord(t, tiles_m, tiles_n);
+        const int ya = tc.m * BM;
+        int yb0, yb1;
+        bool second = true;
+        if (EPI == kEpiSwiGLU) {
+          yb0 = tc.n * 128;
+          yb1 = p.N + tc.n * 128;
+        } else {
+          yb0 = tc.n * BN;
+          yb1 = yb0 + 128;
+          second = yb1 < p.Nb;
+        }
+        const uint32_t bytes = kAStage + (second ? kBStage : kBStage / 2);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&s.empty[stage], phase ^ 1, abort)) {
+            fail(s, p.err);
+            ok = false;
+            break;
+          }
+          const int x = kb * (INT8 ? 128 : 64);
+          mbar_expect_tx(&s.full[stage], bytes);
+          tma_load_2d(s.a + stage * kAStage, &tmA, &s.full[stage], x, ya);
+          tma_load_2d(s.b + stage * kBStage, &tmB, &s.full[stage], x, yb0);
+          if (second) tma_load_2d(s.b + stage * kBStage + kBStage / 2, &tmB, &s.full[stage], x, yb1);
+          ++issued;
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      // Drain: the last loads issued must have landed before the CTA exits.
+      const long outstanding = issued < kStages ? issued : kStages;
+      for (long i = 0; i < outstanding; ++i) {
+        if (--stage < 0) {
+          stage = kStages - 1;
+          phase ^= 1;
+        }
+        mbar_wait(&s.full[stage], phase, nullptr);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = INT8 ? make_idesc(2, 1, BM, BN, false) : make_idesc(1, 1, BM, BN, false);
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++local) {
+        const int buf = local & 1;
+        const uint32_t use = (uint32_t)(local >> 1);
+        if (!mbar_wait(&s.tempty[buf], (use & 1) ^ 1, abort)) {
+          fail(s, p.err);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem_base + buf * BN;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&s.full[stage], phase, abort)) {
+            fail(s, p.err);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(s.a + stage * kAStage);
+          const uint32_t b0 = smem_u32(s.b + stage * kBStage);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint64_t ad = sw128_desc(a0 + k * 32, 16);
+            const uint64_t bd = sw128_desc(b0 + k * 32, 16);
+            if (INT8)
+              mma_s8_ss(d, ad, bd, idesc, (kb | k) != 0);
+            else
+              mma_bf16_ss(d, ad, bd, idesc, (kb | k) != 0);
+          }
+          mma_commit(&s.empty[stage]);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (ok) mma_commit(&s.tfull[buf]);
+      }
+      // every MMA issued by this thread has completed once `drain` flips
+      mma_commit(s.drain);
+      mbar_wait(s.drain, 0, nullptr);
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int quad = warp & 3;
+    int local = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++local) {
+      const TileCoord tc = tile_coord(t, tiles_m, tiles_n);
+      const int buf = local & 1;
+      const uint32_t use = (uint32_t)(local >> 1);
+      if (!mbar_wait(&s.tfull[buf], use & 1, abort)) {
+        if (lane == 0) fail(s, p.err);
+        break;
+      }
+      tc_fence_after();
+      const int64_t row = (int64_t)tc.m * BM + quad * 32 + lane;
+      const uint32_t tacc = tmem_base + ((uint32_t)(quad * 32) << 16) + buf * BN;
+      epilogue_tile<EPI, INT8>(p, tacc, row, row < p.M, tc.n);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.tempty[buf]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
+}
+
+CUresult make_map(PFN_cuTensorMapEncodeTiled_v12000 encode, CUtensorMap* m, const void* ptr, uint64_t rows,
+                  uint64_t cols, bool int8) {
+  const CUtensorMapDataType dt = int8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const uint64_t esz = int8 ? 1 : 2;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * esz};
+  cuuint32_t box[2] = {(cuuint32_t)(kRowBytes / esz), 128};
+  cuuint32_t estr[2] = {1, 1};
+  return encode(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+template <int EPI, bool INT8>
+cudaError_t launch_t(const GemmArgs& a, const CUtensorMap& ta, const CUtensorMap& tb, int num_sms, cudaStream_t s) {
+  auto k = gemm_kernel<EPI, INT8>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const int tiles_m = (int)((a.M + BM - 1) / BM);
+  const int tiles_n = EPI == kEpiSwiGLU ? a.N / 128 : (a.N + BN - 1) / BN;
+  const long tiles = (long)tiles_m * tiles_n;
+  const int grid = (int)(tiles < num_sms ? tiles : num_sms);
+  k<<<grid, kThreads, kSmemBytes, s>>>(ta, tb, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(const GemmArgs& a, PFN_cuTensorMapEncodeTiled_v12000 encode, int num_sms, cudaStream_t s) {
+  if (a.M <= 0) return cudaSuccess;
+  const int kb = a.int8 ? 128 : 64;
+  if (a.K % kb != 0 || a.N % 128 != 0 || a.Nb % 128 != 0) return cudaErrorInvalidValue;
+  if (a.epi == kEpiQKV && (a.head_dim % 32 != 0 || BN % a.head_dim != 0 || a.hd % a.head_dim != 0))
+    return cudaErrorInvalidValue;
+  CUtensorMap ta, tb;
+  if (make_map(encode, &ta, a.A, (uint64_t)a.M, (uint64_t)a.K, a.int8) != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  if (make_map(encode, &tb, a.B, (uint64_t)a.Nb, (uint64_t)a.K, a.int8) != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  if (a.int8) {
+    switch (a.epi) {
+      case kEpiStoreBf16: return launch_t<kEpiStoreBf16, true>(a, ta, tb, num_sms, s);
+      case kEpiQKV: return launch_t<kEpiQKV, true>(a, ta, tb, num_sms, s);
+      case kEpiResid: return launch_t<kEpiResid, true>(a, ta, tb, num_sms, s);
+      case kEpiSwiGLU: return launch_t<kEpiSwiGLU, true>(a, ta, tb, num_sms, s);
+      case kEpiStoreS32: return launch_t<kEpiStoreS32, true>(a, ta, tb, num_sms, s);
+    }
+  } else {
+    switch (a.epi) {
+      case kEpiStoreBf16: return launch_t<kEpiStoreBf16, false>(a, ta, tb, num_sms, s);
+      case kEpiQKV: return launch_t<kEpiQKV, false>(a, ta, tb, num_sms, s);
+      case kEpiResid: return launch_t<kEpiResid, false>(a, ta, tb, num_sms, s);
+      case kEpiSwiGLU: return launch_t<kEpiSwiGLU, false>(a, ta, tb, num_sms, s);
+    }
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace h3

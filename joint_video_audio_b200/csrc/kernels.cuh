@@ -1,0 +1,112 @@
+// Launch interfaces of the block's kernels (internal to libh3blk).
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+namespace h3 {
+
+constexpr int kMaxRopePairs = 128;  // head_dim <= 256
+
+// Rotary table of one head: for pair j, which position axis drives it
+// (0 t, 1 h, 2 w, 3 none) and its frequency.
+struct RopeTable {
+  float freq[kMaxRopePairs];
+  int8_t axis[kMaxRopePairs];
+};
+
+// Per 128-row tile of the packed sequence: number of rows present, number of
+// padding rows among them, and a padding bit per row.
+struct TileInfo {
+  int32_t rows;
+  int32_t npad;
+  uint32_t padbits[4];
+  int32_t _unused[2];
+};
+static_assert(sizeof(TileInfo) == 32, "TileInfo is 32 bytes");
+
+// ---------------------------------------------------------------- prep
+// Validates tag / tidx and fills one TileInfo per 128 rows.
+cudaError_t launch_tile_info(const int32_t* tag, const int32_t* tidx, int64_t n, int n_tags, int n_t,
+                             TileInfo* info, int* err, cudaStream_t s);
+
+// ---------------------------------------------------------------- K1
+// h[r] = rmsnorm(x[r]) * (1 + table[tag][tidx][scale_idx]) + table[..][shift_idx]
+// bf16 output, or (quant) Hadamard-rotated per-token int8 + fp32 scale.
+struct ModNormArgs {
+  const __nv_bfloat16* x;
+  const int32_t* tag;
+  const int32_t* tidx;
+  const float* table;
+  int64_t n;
+  int C, n_tags, n_t, shift_idx, scale_idx;
+  float eps;
+  __nv_bfloat16* out_bf16;  // used when out_q == nullptr
+  int8_t* out_q;
+  float* out_scale;
+};
+cudaError_t launch_modnorm(const ModNormArgs& a, cudaStream_t s);
+
+// ---------------------------------------------------------------- K4
+// Rows of a bf16 matrix [rows, K] -> block-128 Hadamard rotation ->
+// symmetric per-row int8 with fp32 scale.
+cudaError_t launch_rotate_quant(const __nv_bfloat16* in, int64_t rows, int K, int8_t* out_q, float* out_scale,
+                                cudaStream_t s);
+
+// ---------------------------------------------------------------- GEMM
+enum GemmEpilogue : int {
+  kEpiStoreBf16 = 0,  // out = acc
+  kEpiQKV = 1,        // q/k: per-head RMSNorm * gain + RoPE; v: plain
+  kEpiResid = 2,      // out = resid + gate * acc
+  kEpiSwiGLU = 3,     // out[:, j] = silu(acc_gate[:, j]) * acc_up[:, j]
+  kEpiStoreS32 = 4,   // raw int32 accumulators (int8 GEMM only)
+};
+
+struct GemmArgs {
+  // operands: A [M, K] row-major, B [Nb, K] row-major (the weight), both K-major
+  const void* A;
+  const void* B;
+  int64_t M;
+  int N;  // logical output columns (SwiGLU: F)
+  int K;
+  int Nb;  // rows of B
+  bool int8;
+  int epi;
+  // outputs
+  void* out;
+  int64_t ld_out;  // elements
+  // kEpiResid
+  const __nv_bfloat16* resid;
+  const float* table;
+  const int32_t* tag;
+  const int32_t* tidx;
+  int n_tags, n_t, gate_idx;
+  // kEpiQKV
+  const __nv_bfloat16* q_gain;
+  const __nv_bfloat16* k_gain;
+  const int32_t* pos;
+  int head_dim, hd;
+  float qk_eps;
+  RopeTable rope;
+  // int8 dequantisation: acc * s_a[row] * s_b[col]
+  const float* s_a;
+  const float* s_b;
+  int* err;
+};
+cudaError_t launch_gemm(const GemmArgs& a, PFN_cuTensorMapEncodeTiled_v12000 encode, int num_sms, cudaStream_t s);
+
+// ---------------------------------------------------------------- attention
+struct AttnArgs {
+  const __nv_bfloat16* qkv;  // [N, 3*H*D]: q heads, k heads, v heads
+  __nv_bfloat16* o;          // [N, H*D]
+  const int32_t* tag;
+  const TileInfo* tiles;
+  int64_t n;
+  int heads, head_dim;
+  int* err;
+};
+cudaError_t launch_attention(const AttnArgs& a, PFN_cuTensorMapEncodeTiled_v12000 encode, cudaStream_t s);
+
+}  // namespace h3

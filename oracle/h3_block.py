@@ -302,22 +302,12 @@ class BlockOracle:
             out["v"] = self._split_heads(y[:, 2 * HD:])
         return out
 
-    def forward(self, x, tag, tidx, pos, table, rows=None, kv_chunk=4096):
-        """Block forward. ``rows`` (sorted indices) restricts every per-row
-        stage to those query rows; k and v are always computed for all rows,
-        since every query sees every key of its document. Returns a dict of
-        stages for the returned rows: h1, q, k, v, o, x1, h2, a, out (and the
-        full-sequence k, v under "k_all", "v_all")."""
+    def kv_all(self, x, tag, tidx, pos, table, kv_chunk=4096):
+        """k and v ([N, H, D]) of every row of the sequence."""
         d = self.d
         x = f64(x)
-        tag = np.asarray(tag)
-        tidx = np.asarray(tidx)
-        pos = np.asarray(pos)
-        N = x.shape[0]
-        rows = np.arange(N) if rows is None else np.asarray(rows)
         table = f64(table)
-
-        # k, v for every row (in chunks to bound memory)
+        N = x.shape[0]
         k_all = np.empty((N, d.heads, d.head_dim))
         v_all = np.empty((N, d.heads, d.head_dim))
         for s in range(0, N, kv_chunk):
@@ -326,19 +316,37 @@ class BlockOracle:
             h = adaln(x[s:e], m[:, MOD_SHIFT1], m[:, MOD_SCALE1], d.norm_eps)
             kv = self.qkv(h, pos[s:e], part=("k", "v"))
             k_all[s:e], v_all[s:e] = kv["k"], kv["v"]
+        return k_all, v_all
 
-        # per query row
-        m = modulation(table, tag[rows], tidx[rows])
-        xr = x[rows]
+    def query(self, x_rows, tag_rows, tidx_rows, pos_rows, table, k_all, v_all, doc_all):
+        """Every stage of the block for the given query rows, attending to
+        the keys / values of the whole sequence."""
+        d = self.d
+        xr = f64(x_rows)
+        m = modulation(f64(table), tag_rows, tidx_rows)
         h1 = adaln(xr, m[:, MOD_SHIFT1], m[:, MOD_SCALE1], d.norm_eps)
-        q = self.qkv(h1, pos[rows], part=("q",))["q"]
-        doc = documents(tag)
-        o = attention(q, k_all, v_all, doc[rows], doc).reshape(len(rows), d.hd)
+        q = self.qkv(h1, pos_rows, part=("q",))["q"]
+        o = attention(q, k_all, v_all, documents(tag_rows), doc_all).reshape(xr.shape[0], d.hd)
         x1 = xr + m[:, MOD_GATE1] * self.linear(o, "o")
         h2 = adaln(x1, m[:, MOD_SHIFT2], m[:, MOD_SCALE2], d.norm_eps)
         g_u = self.linear(h2, "13")
         a = swiglu(g_u[:, :d.ffn], g_u[:, d.ffn:])
         out = x1 + m[:, MOD_GATE2] * self.linear(a, "2")
-        return {"rows": rows, "h1": h1, "q": q, "k": k_all[rows], "v": v_all[rows],
-                "o": o, "x1": x1, "h2": h2, "a": a, "out": out,
-                "k_all": k_all, "v_all": v_all}
+        return {"h1": h1, "q": q, "o": o, "x1": x1, "h2": h2, "a": a, "out": out}
+
+    def forward(self, x, tag, tidx, pos, table, rows=None, kv_chunk=4096):
+        """Block forward. ``rows`` (sorted indices) restricts every per-row
+        stage to those query rows; k and v are always computed for all rows,
+        since every query sees every key of its document. Returns a dict of
+        stages for the returned rows: h1, q, k, v, o, x1, h2, a, out (and the
+        full-sequence k, v under "k_all", "v_all")."""
+        x = f64(x)
+        tag = np.asarray(tag)
+        tidx = np.asarray(tidx)
+        pos = np.asarray(pos)
+        N = x.shape[0]
+        rows = np.arange(N) if rows is None else np.asarray(rows)
+        k_all, v_all = self.kv_all(x, tag, tidx, pos, table, kv_chunk)
+        r = self.query(x[rows], tag[rows], tidx[rows], pos[rows], table, k_all, v_all, documents(tag))
+        r.update({"rows": rows, "k": k_all[rows], "v": v_all[rows], "k_all": k_all, "v_all": v_all})
+        return r

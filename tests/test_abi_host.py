@@ -1,0 +1,151 @@
+"""Host-side tests of the C-ABI: the library loads, exports every symbol the
+header declares, and rejects bad arguments before touching any GPU."""
+import ctypes as C
+import os
+import re
+import subprocess
+
+import pytest
+
+import h3_inputs as hi
+import joint_video_audio_b200 as j
+from joint_video_audio_b200 import _binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "h3blk.h")
+
+
+def declared_symbols():
+    txt = open(HEADER).read()
+    return sorted(set(re.findall(r"H3BLK_API\s+[\w\s\*]*?\b(h3blk_\w+)\s*\(", txt)))
+
+
+def test_header_declarations_match_binding():
+    assert declared_symbols() == sorted(B.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    out = subprocess.run(["nm", "-D", "--defined-only", B.LIB_PATH], capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (h3blk_\w+)", out))
+    missing = set(declared_symbols()) - exported
+    assert not missing, missing
+    lib = C.CDLL(B.LIB_PATH)
+    for s in declared_symbols():
+        assert getattr(lib, s) is not None
+
+
+def test_version_and_error_strings():
+    assert B.h3blk_version() >= 100
+    for st in range(6):
+        assert B.error_string(st)
+    assert "unknown" in B.error_string(99)
+
+
+def _cfg(**kw):
+    base = dict(hidden=256, heads=6, head_dim=64, ffn=768, n_tags=4, n_t=2, rope_pairs_t=8, rope_pairs_h=12,
+                rope_pairs_w=12, rope_theta=1e4, norm_eps=1e-5, qk_norm_eps=1e-5, quant=0)
+    base.update(kw)
+    return B.h3blk_config(**base)
+
+
+@pytest.mark.parametrize("kw,status", [
+    ({}, B.H3BLK_OK),
+    ({"quant": 1}, B.H3BLK_OK),
+    ({"hidden": 0}, B.H3BLK_ERR_INVALID_ARG),
+    ({"n_t": 0}, B.H3BLK_ERR_INVALID_ARG),
+    ({"rope_theta": -1.0}, B.H3BLK_ERR_INVALID_ARG),
+    ({"quant": 2}, B.H3BLK_ERR_INVALID_ARG),
+    ({"hidden": 200}, B.H3BLK_ERR_UNSUPPORTED),
+    ({"ffn": 700}, B.H3BLK_ERR_UNSUPPORTED),
+    ({"head_dim": 96}, B.H3BLK_ERR_UNSUPPORTED),
+    ({"heads": 3}, B.H3BLK_ERR_UNSUPPORTED),          # 3 * 64 not a multiple of 128
+    ({"rope_pairs_w": 13}, B.H3BLK_ERR_UNSUPPORTED),  # 8 + 12 + 13 > 32
+])
+def test_create_validation(kw, status):
+    assert B.h3blk_create_status(_cfg(**kw)) == status
+
+
+def test_create_null():
+    assert B.h3blk_create_status(None) == B.H3BLK_ERR_INVALID_ARG
+
+
+def test_real_and_page_rope_splits_accepted():
+    # the page's own split: 16 pairs per axis, 96 of 128 channels rotated
+    assert B.h3blk_create_status(_cfg(hidden=5376, heads=56, head_dim=128, ffn=14336,
+                                      rope_pairs_t=16, rope_pairs_h=16, rope_pairs_w=16)) == B.H3BLK_OK
+    assert B.h3blk_create_status(_cfg(hidden=5376, heads=56, head_dim=128, ffn=14336,
+                                      rope_pairs_t=16, rope_pairs_h=24, rope_pairs_w=24)) == B.H3BLK_OK
+
+
+def test_workspace_layout():
+    blk = j.H3Block(hi.REAL)
+    n = 32768
+    ws = blk.workspace_bytes(n)
+    C_, HD, F = 5376, 7168, 14336
+    # h1, qkv, o, x1, h2, a in bf16
+    assert ws >= n * 2 * (C_ + 3 * HD + HD + C_ + C_ + F)
+    assert ws < n * 2 * (C_ + 3 * HD + HD + C_ + C_ + F) + 4 * 1024 * 1024
+    seen = []
+    for name in ("ERROR", "H1", "QKV", "O", "X1", "H2", "A"):
+        off, nb = B.h3blk_stage_view(blk.handle, n, name)
+        assert off % 256 == 0 and off + nb <= ws
+        seen.append((off, off + nb))
+    seen.sort()
+    for (a0, a1), (b0, b1) in zip(seen, seen[1:]):
+        assert a1 <= b0  # no two stages overlap
+    with pytest.raises(B.H3BlkError):
+        B.h3blk_stage_view(blk.handle, n, "H1_Q8")  # not produced by the bf16 path
+    assert blk.workspace_bytes(1) > 0
+    with pytest.raises(B.H3BlkError):
+        B.h3blk_workspace_bytes(blk.handle, 0)
+
+
+def test_w8a8_layout_and_blob():
+    from dataclasses import replace
+    blk = j.H3Block(replace(hi.REAL, quant=1))
+    n = 1000
+    for name in ("H1_Q8", "H1_SCALE", "O_Q8", "O_SCALE", "H2_Q8", "H2_SCALE", "A_Q8", "A_SCALE"):
+        off, nb = B.h3blk_stage_view(blk.handle, n, name)
+        assert off % 256 == 0
+    nb = B.h3blk_int8_weights_bytes(blk.handle)
+    assert nb >= 385351680  # one int8 byte per weight
+
+
+def _fake_forward(blk, n, **override):
+    """A forward call whose pointers are fake host integers: every case here
+    must be rejected by validation before any CUDA call is made."""
+    ws = blk.workspace_bytes(max(n, 1))
+    base = 1 << 40
+    args = dict(x=base, tag=base + (1 << 30), tidx=base + (2 << 30), pos=base + (3 << 30),
+                table=base + (4 << 30), out=base + (5 << 30), ws=base + (6 << 30), ws_bytes=ws)
+    args.update(override)
+    w = B.h3blk_weights(wqkv=base + (8 << 30), q_gain=base + (9 << 30), k_gain=base + (9 << 30) + 256,
+                        wo=base + (10 << 30), w13=base + (11 << 30), w2=base + (12 << 30))
+    return B.h3blk_forward(blk.handle, n, args["x"], args["tag"], args["tidx"], args["pos"], args["table"], w,
+                           args["out"], args["ws"], args["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("override", [
+    {"x": 0}, {"tag": 0}, {"tidx": 0}, {"pos": 0}, {"table": 0}, {"out": 0}, {"ws": 0},
+    {"x": (1 << 40) + 8},              # misaligned
+    {"ws_bytes": 1024},                # workspace too small
+    {"out": 1 << 40},                  # out aliases x
+    {"out": (1 << 40) + (6 << 30)},    # out inside the workspace
+])
+def test_forward_rejects_bad_arguments(override):
+    blk = j.H3Block(hi.TINY)
+    assert _fake_forward(blk, 320, **override) == B.H3BLK_ERR_INVALID_ARG
+
+
+def test_forward_rejects_empty_sequence():
+    blk = j.H3Block(hi.TINY)
+    assert _fake_forward(blk, 0) == B.H3BLK_ERR_INVALID_ARG
+
+
+def test_kernel_level_calls_reject_bad_sizes():
+    assert B.h3blk_rotate_quantize(4, 100, 1 << 40, 1 << 41, 1 << 42, None) == B.H3BLK_ERR_INVALID_ARG
+    assert B.h3blk_rotate_quantize(4, 128 * 200, 1 << 40, 1 << 41, 1 << 42, None) == B.H3BLK_ERR_INVALID_ARG
+    assert B.h3blk_gemm_s8_s32(16, 100, 128, 1 << 40, 1 << 41, 1 << 42, None) == B.H3BLK_ERR_INVALID_ARG
+    assert B.h3blk_gemm_s8_s32(16, 128, 64, 1 << 40, 1 << 41, 1 << 42, None) == B.H3BLK_ERR_INVALID_ARG
+    assert B.h3blk_gemm_bf16(16, 128, 32, 1 << 40, 1 << 41, 1 << 42, None) == B.H3BLK_ERR_INVALID_ARG
+    assert B.h3blk_gemm_bf16(16, 128, 64, 0, 1 << 41, 1 << 42, None) == B.H3BLK_ERR_INVALID_ARG

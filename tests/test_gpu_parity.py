@@ -1,0 +1,190 @@
+"""GPU parity: the CUDA path through the C-ABI against the fp64 oracle and
+against exact / library references, on seeded inputs."""
+from dataclasses import replace
+
+import numpy as np
+import pytest
+import torch
+
+import h3_inputs as hi
+from oracle import h3_block as orc
+from tests._parity import GpuCase, assert_intermediate, assert_stage, errors, to64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    assert torch.cuda.is_available(), "GPU tests need a B200"
+    import joint_video_audio_b200  # noqa: F401  (fails loudly if libh3blk.so is missing)
+    yield
+
+
+# ---------------------------------------------------------------- kernel level
+
+@pytest.mark.parametrize("M,N,K", [(300, 384, 256), (128, 128, 64), (1, 256, 128), (1029, 768, 5376)])
+def test_gemm_bf16_matches_fp32_reference(M, N, K):
+    import joint_video_audio_b200 as j
+    g = torch.Generator().manual_seed(M * 7 + N)
+    a = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    b = (torch.randn(N, K, generator=g) / K ** 0.5).to(torch.bfloat16)
+    c = j.gemm_bf16(a.cuda(), b.cuda())
+    torch.cuda.synchronize()
+    ref = a.double() @ b.double().T
+    assert_stage("gemm_bf16", c, ref)
+
+
+@pytest.mark.parametrize("M,N,K", [(257, 256, 384), (128, 384, 128), (64, 128, 14336)])
+def test_gemm_s8_exact(M, N, K):
+    import joint_video_audio_b200 as j
+    g = torch.Generator().manual_seed(M + N + K)
+    a = torch.randint(-127, 128, (M, K), generator=g, dtype=torch.int8)
+    b = torch.randint(-127, 128, (N, K), generator=g, dtype=torch.int8)
+    c = j.gemm_s8_s32(a.cuda(), b.cuda()).cpu()
+    ref = orc.int8_matmul_exact(a.numpy(), b.numpy())
+    assert np.array_equal(c.numpy().astype(np.int64), ref)
+
+
+def test_gemm_s8_extreme_values_exact():
+    import joint_video_audio_b200 as j
+    K = 14336
+    a = torch.full((128, K), 127, dtype=torch.int8)
+    a[1] = -127
+    b = torch.full((128, K), 127, dtype=torch.int8)
+    c = j.gemm_s8_s32(a.cuda(), b.cuda()).cpu()
+    assert int(c[0, 0]) == 231225344 and int(c[1, 5]) == -231225344
+
+
+@pytest.mark.parametrize("rows,K", [(5, 256), (33, 7168), (17, 14336), (3, 5376)])
+def test_rotate_quantize_vs_oracle(rows, K):
+    import joint_video_audio_b200 as j
+    g = torch.Generator().manual_seed(rows * K)
+    x = (torch.randn(rows, K, generator=g) * 0.7).to(torch.bfloat16)
+    x[0] = 0  # amax = 0 row
+    q, s = j.rotate_quantize(x.cuda())
+    q, s = q.cpu().numpy().astype(np.int64), s.cpu().numpy().astype(np.float64)
+    rq, rs = orc.quantize_rows(orc.rotate_blocks(x))
+    assert np.all(q[0] == 0) and s[0] == 0
+    np.testing.assert_allclose(s, rs, rtol=1e-5)
+    d = np.abs(q - rq.astype(np.int64))
+    assert d.max() <= 1
+    assert np.mean(d == 0) >= 0.999
+
+
+# ---------------------------------------------------------------- tiny block
+
+@pytest.fixture(scope="module")
+def tiny():
+    inp = hi.make_inputs("tiny_320")
+    case = GpuCase(inp)
+    case.run()
+    lay = inp.layout
+    ref = orc.BlockOracle(inp.dims, inp.weights).forward(inp.x, lay.tag, lay.tidx, lay.pos, inp.table)
+    return case, ref
+
+
+def test_tiny_stage_h1(tiny):
+    case, ref = tiny
+    assert_intermediate("h1", case.stage("H1"), ref["h1"])
+
+
+def test_tiny_stage_qkv(tiny):
+    case, ref = tiny
+    q, k, v = case.qkv()
+    assert_intermediate("q", q, ref["q"])
+    assert_intermediate("k", k, ref["k"])
+    assert_intermediate("v", v, ref["v"])
+
+
+def test_tiny_stage_attention(tiny):
+    case, ref = tiny
+    assert_intermediate("o", case.stage("O"), ref["o"])
+
+
+def test_tiny_stages_x1_h2_a_out(tiny):
+    case, ref = tiny
+    assert_intermediate("x1", case.stage("X1"), ref["x1"])
+    assert_intermediate("h2", case.stage("H2"), ref["h2"])
+    assert_intermediate("a", case.stage("A"), ref["a"])
+    assert_stage("out", case.out, ref["out"])
+
+
+def test_tiny_padding_rows_unchanged_and_isolated(tiny):
+    case, ref = tiny
+    pad = torch.from_numpy(case.inp.layout.tag == -1).cuda()
+    out0 = case.run().clone()
+    assert torch.equal(out0[pad], case.x[pad])
+    x2 = case.x.clone()
+    x2[pad] = (torch.randn(int(pad.sum()), case.dims.hidden, device="cuda") * 7).to(torch.bfloat16)
+    out1 = case.run(x=x2).clone()
+    assert torch.equal(out1[~pad], out0[~pad])
+    assert torch.equal(out1[pad], x2[pad])
+    case.run()
+
+
+def test_tiny_zero_gates_identity(tiny):
+    case, _ = tiny
+    t = case.table.clone()
+    t[:, :, 2] = 0
+    t[:, :, 5] = 0
+    out = case.run(table=t).clone()
+    assert torch.equal(out, case.x)
+    case.run()
+
+
+def test_tiny_bad_index_reported():
+    import joint_video_audio_b200 as j
+    inp = hi.make_inputs("tiny_320")
+    case = GpuCase(inp)
+    case.tag[3] = 9  # outside n_tags
+    case.run()
+    assert case.block.check(case.ws, case.n) == j.capi.H3BLK_ERR_BAD_INDEX
+    case.tag[3] = 0
+    case.tidx[5] = -3
+    case.run()
+    assert case.block.check(case.ws, case.n) == j.capi.H3BLK_ERR_BAD_INDEX
+    case.tidx[5] = 0
+    case.run()
+    assert case.block.check(case.ws, case.n) == j.capi.H3BLK_OK
+
+
+@pytest.mark.parametrize("n", [1, 2, 127, 129, 255, 300])
+def test_tiny_ragged_lengths(n):
+    full = hi.layout_tiny()
+    n_pad = n // 4  # the tail keeps some padding rows
+    sel = np.r_[np.arange(n - n_pad), np.arange(full.n - n_pad, full.n)]
+    lay = hi.Layout(f"tiny_{n}", full.tag[sel], full.tidx[sel], full.pos[sel])
+    inp = hi.make_inputs(hi.TINY, lay)
+    case = GpuCase(inp)
+    case.run()
+    ref = orc.BlockOracle(inp.dims, inp.weights).forward(inp.x, lay.tag, lay.tidx, lay.pos, inp.table)
+    assert_intermediate("o", case.stage("O"), ref["o"])
+    assert_stage("out", case.out, ref["out"])
+
+
+def test_tiny_padding_anywhere():
+    base = hi.layout_tiny()
+    perm = np.random.default_rng(5).permutation(base.n)
+    lay = hi.Layout("tiny_perm", base.tag[perm], base.tidx[perm], base.pos[perm])
+    inp = hi.make_inputs(hi.TINY, lay)
+    case = GpuCase(inp)
+    case.run()
+    ref = orc.BlockOracle(inp.dims, inp.weights).forward(inp.x, lay.tag, lay.tidx, lay.pos, inp.table)
+    assert_intermediate("o", case.stage("O"), ref["o"])
+    assert_stage("out", case.out, ref["out"])
+
+
+def test_tiny_w8a8_block():
+    inp = hi.make_inputs("tiny_320")
+    inp.dims = replace(inp.dims, quant=1)
+    case = GpuCase(inp)
+    case.run()
+    lay = inp.layout
+    ob = orc.BlockOracle(inp.dims, inp.weights)
+    ref = ob.forward(inp.x, lay.tag, lay.tidx, lay.pos, inp.table)
+    q, k, v = case.qkv()
+    assert_intermediate("q", q, ref["q"])
+    assert_intermediate("k", k, ref["k"])
+    assert_intermediate("o", case.stage("O"), ref["o"])
+    assert_intermediate("a", case.stage("A"), ref["a"], rel_rms=2e-2)
+    assert_stage("out", case.out, ref["out"])
