@@ -5,19 +5,32 @@
 // in their own attention document by a boolean mask. The attention scale is
 // 1/sqrt(head_dim).
 //
-// One CTA per (128-query tile, head). Roles:
-//   warp 0      TMA: Q once; lane 0 streams K tiles, lane 1 streams V tiles
-//               (two stages each, so K loads never wait on a P*V product)
-//   warp 1      TMEM allocator + single-thread MMA issuer:
-//                 S[j%2] = Q K_j^T            (M=128, N=128, K=head_dim)
-//                 O     += P_{j-1} V_{j-1}    (M=128, N=head_dim, K=128)
-//   warps 2..5  softmax, one thread per query row: S row from TMEM, mask,
-//               online max / sum in the exp2 domain, P (bf16) into shared
-//               memory in the swizzled K-major layout the MMA reads, and the
-//               rescale of O in TMEM when the running max grows by more than
-//               2^8 (otherwise the stale max is kept: values stay below 256).
-// KV tiles whose rows all lie in the other document are skipped; tiles that
-// mix documents, or run past the end of the sequence, are masked per element.
+// One CTA per (pair of 128-query tiles, head). The two query tiles ping-pong:
+// while the softmax warps of one tile work, the tensor core runs the other
+// tile's products, so the exponentials overlap the MMAs.
+//
+//   warp 0      TMA: both Q tiles once, then K_0, V_0, K_1, V_1, ... through a
+//               ring of shared-memory slots
+//   warp 1      TMEM allocator + single-thread MMA issuer, in the order
+//                 S0_0 S1_0 | PV0_0 S0_1 PV1_0 S1_1 | PV0_1 S0_2 PV1_1 S1_2 | ...
+//               with Sq_j = Qq K_j^T (M=128, N=128, K=head_dim) and
+//               PVq_j: Oq += Pq_j V_j (M=128, N=head_dim, K=128)
+//   warps 2..5  softmax of query tile 0, warps 6..9 of query tile 1; one
+//               thread per query row: S row from TMEM, mask, online max / sum
+//               in the exp2 domain, P (bf16) into shared memory in the
+//               swizzled K-major layout the MMA reads, and the rescale of O in
+//               TMEM when the running max grows by more than 2^8 (otherwise the
+//               stale max is kept, so P stays below 256).
+// The two query tiles share one P buffer: P1_j is written once P0_j V_j has
+// completed and P0_{j+1} once P1_j V_j has, which the MMA order above allows
+// without a bubble (an S product runs in between). That frees shared memory
+// for a four-slot K/V ring, so K_{j+1} and V_{j+1} are fetched one full
+// iteration ahead.
+// Tensor memory: S0 | S1 | O0 | O1 (128 columns each).
+// KV tiles whose rows all lie in the other document are skipped when neither
+// query tile needs them; tiles that mix documents, run past the end of the
+// sequence, or belong to the other document of one of the two query tiles are
+// masked per element.
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 #include <math_constants.h>
@@ -28,51 +41,45 @@
 namespace h3 {
 namespace {
 
-constexpr int kThreads = 192;
 constexpr int kTile = 128;
-constexpr uint32_t kTmemCols = 512;  // S0 | S1 | O
+constexpr int kSoftmaxWarps = 8;
+constexpr int kThreads = 32 * (2 + kSoftmaxWarps);
+constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;
 
 template <int D>
 struct AttnSmem {
-  static constexpr int kQBytes = kTile * D * 2;
-  static constexpr int kKVBytes = kTile * D * 2;
-  static constexpr int kPBytes = kTile * kTile * 2;
-  static constexpr int kRegion = kTile * 128;  // one 128-row x 128-byte swizzle region
-  static constexpr size_t kBytes = 1024 + kQBytes + 4 * (size_t)kKVBytes + kPBytes + 256;
-  uint8_t *q, *k[2], *v[2], *p;
-  uint64_t *q_full, *k_full, *k_empty, *v_full, *v_empty, *s_full, *s_free, *p_full, *o_ready, *o_final;
+  static constexpr int kSlots = D == 128 ? 4 : 8;
+  static constexpr int kQBytes = kTile * D * 2;     // one query tile
+  static constexpr int kKVBytes = kTile * D * 2;    // one K or V tile
+  static constexpr int kPBytes = kTile * kTile * 2; // one P tile
+  static constexpr int kRegion = kTile * 128;       // 128 rows x 128 bytes (one swizzle region)
+  static constexpr size_t kBytes = 1024 + 2 * (size_t)kQBytes + (size_t)kPBytes + kSlots * (size_t)kKVBytes + 512;
+  uint8_t *q0, *p, *slot0;  // query tile t at q0 + t * kQBytes, ring slot i at slot0 + i * kKVBytes
+  uint64_t *q_full, *ring_full, *ring_empty, *s_full, *s_free, *p_full, *o_ready, *o_final;
   uint32_t* tmem_base;
   int* abort;
 
   __device__ explicit AttnSmem(uint8_t* raw) {
     const uint32_t base = smem_u32(raw);
     uint8_t* x = raw + (((base + 1023u) & ~1023u) - base);
-    q = x;
-    x += kQBytes;
-    for (int i = 0; i < 2; ++i) {
-      k[i] = x;
-      x += kKVBytes;
-    }
-    for (int i = 0; i < 2; ++i) {
-      v[i] = x;
-      x += kKVBytes;
-    }
+    q0 = x;
+    x += 2 * kQBytes;
     p = x;
     x += kPBytes;
+    slot0 = x;
+    x += kSlots * kKVBytes;
     uint64_t* b = reinterpret_cast<uint64_t*>(x);
     q_full = b;
-    k_full = b + 1;
-    k_empty = b + 3;
-    v_full = b + 5;
-    v_empty = b + 7;
-    s_full = b + 9;
-    s_free = b + 11;
-    p_full = b + 13;
-    o_ready = b + 14;
-    o_final = b + 15;
-    tmem_base = reinterpret_cast<uint32_t*>(b + 16);
-    abort = reinterpret_cast<int*>(b + 17);
+    ring_full = b + 1;
+    ring_empty = b + 1 + kSlots;
+    s_full = b + 1 + 2 * kSlots;
+    s_free = s_full + 2;
+    p_full = s_full + 4;
+    o_ready = s_full + 6;
+    o_final = s_full + 8;
+    tmem_base = reinterpret_cast<uint32_t*>(s_full + 9);
+    abort = reinterpret_cast<int*>(s_full + 10);
   }
 };
 
@@ -81,14 +88,25 @@ __device__ __forceinline__ int tile_kind(const TileInfo& t) {
   return t.npad == 0 ? 0 : (t.npad == t.rows ? 1 : 2);
 }
 
-// Advances `kt` to the next KV tile that the query tile must visit.
-__device__ __forceinline__ int next_kv_tile(const TileInfo* tiles, int n_tiles, int qkind, int kt) {
+__device__ __forceinline__ bool skips(int qkind, int kkind) {
+  return (qkind == 0 && kkind == 1) || (qkind == 1 && kkind == 0);
+}
+
+// Next KV tile at or after kt that at least one of the two query tiles needs.
+__device__ __forceinline__ int next_kv_tile(const TileInfo* tiles, int n_tiles, int qk0, int qk1, int kt) {
   for (; kt < n_tiles; ++kt) {
     const int kk = tile_kind(tiles[kt]);
-    if ((qkind == 0 && kk == 1) || (qkind == 1 && kk == 0)) continue;
-    return kt;
+    if (!(skips(qk0, kk) && skips(qk1, kk))) return kt;
   }
   return n_tiles;
+}
+
+__device__ __forceinline__ int count_kv_tiles(const TileInfo* tiles, int n_tiles, int qk0, int qk1) {
+  int n = 0;
+  for (int kt = next_kv_tile(tiles, n_tiles, qk0, qk1, 0); kt < n_tiles;
+       kt = next_kv_tile(tiles, n_tiles, qk0, qk1, kt + 1))
+    ++n;
+  return n;
 }
 
 __device__ __forceinline__ void fail(int* err, volatile int* abort) {
@@ -99,28 +117,32 @@ __device__ __forceinline__ void fail(int* err, volatile int* abort) {
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant__ CUtensorMap tm, const AttnArgs p) {
   extern __shared__ uint8_t smem_raw[];
-  AttnSmem<D> s(smem_raw);
   using SM = AttnSmem<D>;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = blockIdx.x, head = blockIdx.y;
-  const int n_tiles = (int)((p.n + kTile - 1) / kTile);
-  const int HD = p.heads * D;
-  const int qkind = tile_kind(p.tiles[qt]);
-  volatile int* abort = s.abort;
+  SM s(smem_raw);
+  constexpr int kSlots = SM::kSlots;
   constexpr int kRegions = D / 64;  // 64-column swizzle regions of a Q/K/V tile
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int pair = blockIdx.x, head = blockIdx.y;
+  const int n_tiles = (int)((p.n + kTile - 1) / kTile);
+  const int qt0 = 2 * pair;
+  const int HD = p.heads * D;
+  // a missing second tile (odd tile count) behaves like an all-valid tile
+  const int qk0 = tile_kind(p.tiles[qt0]);
+  const int qk1 = qt0 + 1 < n_tiles ? tile_kind(p.tiles[qt0 + 1]) : 0;
+  volatile int* abort = s.abort;
 
   if (threadIdx.x == 0) {
     mbar_init(s.q_full, 1);
+    for (int i = 0; i < kSlots; ++i) {
+      mbar_init(&s.ring_full[i], 1);
+      mbar_init(&s.ring_empty[i], 1);
+    }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&s.k_full[i], 1);
-      mbar_init(&s.k_empty[i], 1);
-      mbar_init(&s.v_full[i], 1);
-      mbar_init(&s.v_empty[i], 1);
       mbar_init(&s.s_full[i], 1);
       mbar_init(&s.s_free[i], 4);
+      mbar_init(&s.p_full[i], 4);
+      mbar_init(&s.o_ready[i], 1);
     }
-    mbar_init(s.p_full, 4);
-    mbar_init(s.o_ready, 1);
     mbar_init(s.o_final, 1);
     *s.abort = 0;
     fence_mbar_init();
@@ -133,89 +155,101 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *s.tmem_base;
-  const uint32_t t_s = tmem, t_o = tmem + 256;
+  const int n_kv = count_kv_tiles(p.tiles, n_tiles, qk0, qk1);
 
   if (warp == 0) {
     // ------------------------------------------------------------ loads
     if (lane == 0) {
       tma_prefetch_desc(&tm);
-      mbar_expect_tx(s.q_full, SM::kQBytes);
-      for (int r = 0; r < kRegions; ++r)
-        tma_load_2d(s.q + r * SM::kRegion, &tm, s.q_full, head * D + r * 64, qt * kTile);
-    }
-    if (lane == 0 || lane == 1) {
-      const bool is_k = lane == 0;
-      uint64_t* full = is_k ? s.k_full : s.v_full;
-      uint64_t* empty = is_k ? s.k_empty : s.v_empty;
-      const int col = (is_k ? HD : 2 * HD) + head * D;
-      int j = 0;
-      for (int kt = next_kv_tile(p.tiles, n_tiles, qkind, 0); kt < n_tiles;
-           kt = next_kv_tile(p.tiles, n_tiles, qkind, kt + 1), ++j) {
-        const int st = j & 1;
-        if (!mbar_wait(&empty[st], ((j >> 1) & 1) ^ 1, abort)) {
-          fail(p.err, abort);
-          break;
+      // a second query tile past the end of the sequence is not loaded: its
+      // rows are never stored
+      const int nq = qt0 + 1 < n_tiles ? 2 : 1;
+      mbar_expect_tx(s.q_full, nq * SM::kQBytes);
+      for (int t = 0; t < nq; ++t)
+        for (int r = 0; r < kRegions; ++r)
+          tma_load_2d(s.q0 + t * SM::kQBytes + r * SM::kRegion, &tm, s.q_full, head * D + r * 64, (qt0 + t) * kTile);
+      int u = 0;
+      for (int kt = next_kv_tile(p.tiles, n_tiles, qk0, qk1, 0); kt < n_tiles;
+           kt = next_kv_tile(p.tiles, n_tiles, qk0, qk1, kt + 1)) {
+        bool ok = true;
+        for (int kv = 0; kv < 2; ++kv, ++u) {  // K_j then V_j
+          const int sl = u % kSlots;
+          if (!mbar_wait(&s.ring_empty[sl], ((u / kSlots) & 1) ^ 1, abort)) {
+            fail(p.err, abort);
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(&s.ring_full[sl], SM::kKVBytes);
+          const int col = (kv == 0 ? HD : 2 * HD) + head * D;
+          for (int r = 0; r < kRegions; ++r)
+            tma_load_2d(s.slot0 + sl * SM::kKVBytes + r * SM::kRegion, &tm, &s.ring_full[sl], col + r * 64, kt * kTile);
         }
-        uint8_t* dst = is_k ? s.k[st] : s.v[st];
-        mbar_expect_tx(&full[st], SM::kKVBytes);
-        for (int r = 0; r < kRegions; ++r) tma_load_2d(dst + r * SM::kRegion, &tm, &full[st], col + r * 64, kt * kTile);
+        if (!ok) break;
       }
-      // drain the last (up to two) loads before the CTA may exit
-      for (int i = 0; i < 2 && j - 1 - i >= 0; ++i) {
-        const int jj = j - 1 - i;
-        mbar_wait(&full[jj & 1], (jj >> 1) & 1, nullptr);
+      // drain: the last loads must land before the CTA may exit
+      for (int i = 0; i < kSlots && u - 1 - i >= 0; ++i) {
+        const int uu = u - 1 - i;
+        mbar_wait(&s.ring_full[uu % kSlots], (uu / kSlots) & 1, nullptr);
       }
+      mbar_wait(s.q_full, 0, nullptr);
     }
-    if (lane == 0) mbar_wait(s.q_full, 0, nullptr);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA
     if (lane == 0) {
       constexpr uint32_t idesc_qk = make_idesc(1, 1, kTile, kTile, false);
       constexpr uint32_t idesc_pv = make_idesc(1, 1, kTile, D, true);
-      const uint32_t q0 = smem_u32(s.q), p0 = smem_u32(s.p);
-      bool ok = mbar_wait(s.q_full, 0, abort);
-      int j = 0;
-      auto issue_pv = [&](int i) -> bool {
-        const int st = i & 1;
-        if (!mbar_wait(s.p_full, i & 1, abort)) return false;
-        if (!mbar_wait(&s.v_full[st], (i >> 1) & 1, abort)) return false;
+      const uint32_t q0 = smem_u32(s.q0), ring0 = smem_u32(s.slot0);
+      auto slot_of = [](int u) { return u % kSlots; };
+      auto wait_ring = [&](int u) { return mbar_wait(&s.ring_full[u % kSlots], (u / kSlots) & 1, abort); };
+      // S_t = Q_t K_j^T into TMEM columns [t*128, t*128+128)
+      auto issue_s = [&](int t, int j) -> bool {
+        if (j > 0 && !mbar_wait(&s.s_free[t], (j - 1) & 1, abort)) return false;
         tc_fence_after();
-        const uint32_t v0 = smem_u32(s.v[st]);
+        const uint32_t qa = q0 + t * SM::kQBytes;
+        const uint32_t ka = ring0 + slot_of(2 * j) * SM::kKVBytes;
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk) {
-          const uint64_t ad = sw128_desc(p0 + (kk >> 2) * SM::kRegion + (kk & 3) * 32, 16);
-          const uint64_t bd = sw128_desc(v0 + kk * 16 * 128, SM::kRegion);
-          mma_bf16_ss(t_o, ad, bd, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * SM::kRegion + (kk & 3) * 32;
+          mma_bf16_ss(tmem + t * kTile, sw128_desc(qa + off, 16), sw128_desc(ka + off, 16), idesc_qk,
+                      kk > 0 ? 1u : 0u);
         }
-        mma_commit(&s.v_empty[st]);
-        mma_commit(s.o_ready);
+        mma_commit(&s.s_full[t]);
         return true;
       };
-      if (ok) {
-        for (int kt = next_kv_tile(p.tiles, n_tiles, qkind, 0); kt < n_tiles;
-             kt = next_kv_tile(p.tiles, n_tiles, qkind, kt + 1), ++j) {
-          const int st = j & 1;
-          if (!mbar_wait(&s.k_full[st], (j >> 1) & 1, abort) ||
-              !mbar_wait(&s.s_free[st], ((j >> 1) & 1) ^ 1, abort)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t k0 = smem_u32(s.k[st]);
+      // O_t += P_t V_j into TMEM columns [256 + t*128, ...)
+      auto issue_pv = [&](int t, int j) -> bool {
+        if (!mbar_wait(&s.p_full[t], j & 1, abort)) return false;
+        tc_fence_after();
+        const uint32_t pa = smem_u32(s.p);
+        const uint32_t va = ring0 + slot_of(2 * j + 1) * SM::kKVBytes;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * SM::kRegion + (kk & 3) * 32;
-            mma_bf16_ss(t_s + st * kTile, sw128_desc(q0 + off, 16), sw128_desc(k0 + off, 16), idesc_qk,
-                        kk > 0 ? 1u : 0u);
-          }
-          mma_commit(&s.k_empty[st]);
-          mma_commit(&s.s_full[st]);
-          if (j > 0 && !issue_pv(j - 1)) {
-            ok = false;
-            break;
+        for (int kk = 0; kk < kTile / 16; ++kk) {
+          const uint64_t ad = sw128_desc(pa + (kk >> 2) * SM::kRegion + (kk & 3) * 32, 16);
+          const uint64_t bd = sw128_desc(va + kk * 16 * 128, SM::kRegion);
+          mma_bf16_ss(tmem + 256 + t * kTile, ad, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&s.o_ready[t]);
+        return true;
+      };
+      bool ok = mbar_wait(s.q_full, 0, abort);
+      if (ok && n_kv > 0) {
+        ok = wait_ring(0) && issue_s(0, 0) && issue_s(1, 0);
+        if (ok) mma_commit(&s.ring_empty[slot_of(0)]);
+        for (int j = 0; ok && j < n_kv; ++j) {
+          ok = wait_ring(2 * j + 1) && issue_pv(0, j);
+          if (!ok) break;
+          const bool more = j + 1 < n_kv;
+          if (more) ok = wait_ring(2 * j + 2) && issue_s(0, j + 1);
+          if (!ok) break;
+          ok = issue_pv(1, j);
+          if (!ok) break;
+          mma_commit(&s.ring_empty[slot_of(2 * j + 1)]);
+          if (more) {
+            ok = issue_s(1, j + 1);
+            if (!ok) break;
+            mma_commit(&s.ring_empty[slot_of(2 * j + 2)]);
           }
         }
-        if (ok && j > 0) ok = issue_pv(j - 1);
       }
       if (!ok) fail(p.err, abort);
       mma_commit(s.o_final);
@@ -223,63 +257,78 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     }
   } else {
     // ------------------------------------------------------------ softmax
+    const int t = (warp - 2) >> 2;  // query tile of this warpgroup
     const int quad = warp & 3;
     const int r = quad * 32 + lane;  // row within the tile = TMEM lane
+    const int qt = qt0 + t;
     const int64_t row = (int64_t)qt * kTile + r;
     const bool row_ok = row < p.n;
     const uint32_t my_pad = (row_ok && p.tag[row] == -1) ? 1u : 0u;
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+    const uint32_t t_s = tmem + lane_base + t * kTile;
+    const uint32_t t_o = tmem + lane_base + 256 + t * kTile;
     const float scale_log2 = 1.4426950408889634f * rsqrtf((float)D);
+    const int myk = t == 0 ? qk0 : qk1;
     float m_run = -CUDART_INF_F, l_run = 0.f;
     uint8_t* prow = s.p + r * 128;
     bool ok = true;
     int j = 0;
-    for (int kt = next_kv_tile(p.tiles, n_tiles, qkind, 0); kt < n_tiles;
-         kt = next_kv_tile(p.tiles, n_tiles, qkind, kt + 1), ++j) {
-      const int sb = j & 1;
-      if (!mbar_wait(&s.s_full[sb], (j >> 1) & 1, abort)) {
+    for (int kt = next_kv_tile(p.tiles, n_tiles, qk0, qk1, 0); kt < n_tiles;
+         kt = next_kv_tile(p.tiles, n_tiles, qk0, qk1, kt + 1), ++j) {
+      if (!mbar_wait(&s.s_full[t], j & 1, abort)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      float sv[kTile];
-#pragma unroll
-      for (int c = 0; c < kTile / 32; ++c) {
-        uint32_t u[32];
-        tmem_ld32(t_s + lane_base + sb * kTile + c * 32, u);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) sv[c * 32 + i] = __uint_as_float(u[i]);
-      }
+      uint32_t u[kTile];
+      tmem_ld128(t_s, u);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s.s_free[sb]);
-
-      const TileInfo ti = p.tiles[kt];
-      const bool masked = !(tile_kind(ti) == qkind && qkind != 2) || ti.rows < kTile;
-      if (masked) {
+      if (lane == 0) mbar_arrive(&s.s_free[t]);
+      float* sv = reinterpret_cast<float*>(u);
+      {
+        const TileInfo& ti = p.tiles[kt];
+        const int kk = tile_kind(ti);
+        if (!(kk == myk && myk != 2) || ti.rows < kTile) {
+          const int rows = ti.rows;
 #pragma unroll
-        for (int c = 0; c < kTile; ++c) {
-          const uint32_t pad = (ti.padbits[c >> 5] >> (c & 31)) & 1u;
-          if (c >= ti.rows || pad != my_pad) sv[c] = -CUDART_INF_F;
+          for (int w = 0; w < 4; ++w) {
+            const uint32_t bits = ti.padbits[w] ^ (my_pad ? 0xffffffffu : 0u);  // 1 = other document
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              if (((bits >> c) & 1u) || w * 32 + c >= rows) sv[w * 32 + c] = -CUDART_INF_F;
+          }
         }
       }
-      float mx = -CUDART_INF_F;
+      float mx0 = -CUDART_INF_F, mx1 = -CUDART_INF_F;
 #pragma unroll
-      for (int c = 0; c < kTile; ++c) mx = fmaxf(mx, sv[c]);
-      mx *= scale_log2;
-      const float m_new = fmaxf(m_run, mx);
+      for (int c = 0; c < kTile; c += 2) {
+        mx0 = fmaxf(mx0, sv[c]);
+        mx1 = fmaxf(mx1, sv[c + 1]);
+      }
+      const float m_new = fmaxf(m_run, fmaxf(mx0, mx1) * scale_log2);
       const bool grow = m_new > m_run + kRescaleThreshold || (m_run == -CUDART_INF_F && m_new != -CUDART_INF_F);
       const float m_use = grow ? m_new : m_run;
       const float m_sub = m_use == -CUDART_INF_F ? 0.f : m_use;
       const float alpha = grow ? ex2_approx(m_run - m_use) : 1.f;
-      float rs = 0.f;
+      float rs0 = 0.f, rs1 = 0.f;
+      // exponentials, packed to bf16 pairs in place: u[0..63] holds P's row
 #pragma unroll
-      for (int c = 0; c < kTile; ++c) {
-        sv[c] = ex2_approx(fmaf(sv[c], scale_log2, -m_sub));
-        rs += sv[c];
+      for (int c = 0; c < kTile; c += 2) {
+        const float e0 = ex2_approx(fmaf(sv[c], scale_log2, -m_sub));
+        const float e1 = ex2_approx(fmaf(sv[c + 1], scale_log2, -m_sub));
+        rs0 += e0;
+        rs1 += e1;
+        u[c >> 1] = pack_bf16x2(e0, e1);
       }
-      // P_{j-1} V_{j-1} must be complete: the P buffer is reused and O may be rescaled
-      if (j > 0 && !mbar_wait(s.o_ready, (j - 1) & 1, abort)) {
+      // O may be rescaled once this tile's previous P V has completed; the
+      // shared P buffer is free once the other tile's latest P V has
+      if (j > 0 && !mbar_wait(&s.o_ready[t], (j - 1) & 1, abort)) {
+        ok = false;
+        break;
+      }
+      if (t == 0 ? (j > 0 && !mbar_wait(&s.o_ready[1], (j - 1) & 1, abort))
+                 : !mbar_wait(&s.o_ready[0], j & 1, abort)) {
         ok = false;
         break;
       }
@@ -287,31 +336,27 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         tc_fence_after();
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
-          uint32_t u[32];
-          tmem_ld32(t_o + lane_base + c * 32, u);
+          uint32_t o[32];
+          tmem_ld32(t_o + c * 32, o);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
-          tmem_st32(t_o + lane_base + c * 32, u);
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(t_o + c * 32, o);
         }
         tmem_wait_st();
       }
-      l_run = l_run * alpha + rs;
+      l_run = l_run * alpha + (rs0 + rs1);
       m_run = m_use;
       // P row -> shared memory, 128-byte swizzle, two 64-column regions
 #pragma unroll
       for (int c = 0; c < kTile / 8; ++c) {
-        uint4 w;
-        w.x = pack_bf16x2(sv[8 * c + 0], sv[8 * c + 1]);
-        w.y = pack_bf16x2(sv[8 * c + 2], sv[8 * c + 3]);
-        w.z = pack_bf16x2(sv[8 * c + 4], sv[8 * c + 5]);
-        w.w = pack_bf16x2(sv[8 * c + 6], sv[8 * c + 7]);
         const int region = c >> 3, cc = c & 7;
-        *reinterpret_cast<uint4*>(prow + region * SM::kRegion + ((cc ^ (r & 7)) << 4)) = w;
+        *reinterpret_cast<uint4*>(prow + region * SM::kRegion + ((cc ^ (r & 7)) << 4)) =
+            make_uint4(u[4 * c], u[4 * c + 1], u[4 * c + 2], u[4 * c + 3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(s.p_full);
+      if (lane == 0) mbar_arrive(&s.p_full[t]);
     }
     if (!ok) {
       if (lane == 0) fail(p.err, abort);
@@ -321,17 +366,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       __nv_bfloat16* dst = p.o + row * (int64_t)HD + head * D;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
-        uint32_t u[32];
-        tmem_ld32(t_o + lane_base + c * 32, u);
+        uint32_t o[32];
+        tmem_ld32(t_o + c * 32, o);
         if (row_ok) {
           uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(u[8 * i + 0]) * inv_l, __uint_as_float(u[8 * i + 1]) * inv_l);
-            w.y = pack_bf16x2(__uint_as_float(u[8 * i + 2]) * inv_l, __uint_as_float(u[8 * i + 3]) * inv_l);
-            w.z = pack_bf16x2(__uint_as_float(u[8 * i + 4]) * inv_l, __uint_as_float(u[8 * i + 5]) * inv_l);
-            w.w = pack_bf16x2(__uint_as_float(u[8 * i + 6]) * inv_l, __uint_as_float(u[8 * i + 7]) * inv_l);
+            w.x = pack_bf16x2(__uint_as_float(o[8 * i + 0]) * inv_l, __uint_as_float(o[8 * i + 1]) * inv_l);
+            w.y = pack_bf16x2(__uint_as_float(o[8 * i + 2]) * inv_l, __uint_as_float(o[8 * i + 3]) * inv_l);
+            w.z = pack_bf16x2(__uint_as_float(o[8 * i + 4]) * inv_l, __uint_as_float(o[8 * i + 5]) * inv_l);
+            w.w = pack_bf16x2(__uint_as_float(o[8 * i + 6]) * inv_l, __uint_as_float(o[8 * i + 7]) * inv_l);
             d4[i] = w;
           }
         }
@@ -352,7 +397,8 @@ cudaError_t launch_d(const AttnArgs& a, const CUtensorMap& tm, cudaStream_t s) {
   auto k = attn_kernel<D>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)AttnSmem<D>::kBytes);
   if (e != cudaSuccess) return e;
-  const dim3 grid((unsigned)((a.n + kTile - 1) / kTile), (unsigned)a.heads);
+  const int n_tiles = (int)((a.n + kTile - 1) / kTile);
+  const dim3 grid((unsigned)((n_tiles + 1) / 2), (unsigned)a.heads);
   k<<<grid, kThreads, AttnSmem<D>::kBytes, s>>>(tm, a);
   return cudaGetLastError();
 }
