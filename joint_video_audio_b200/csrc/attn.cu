@@ -46,6 +46,7 @@ constexpr int kSoftmaxWarps = 8;
 constexpr int kThreads = 32 * (2 + kSoftmaxWarps);
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;
+constexpr int kPolyEvery = 4;  // one exponential pair in four on the FMA pipe
 
 template <int D>
 struct AttnSmem {
@@ -300,27 +301,45 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
           }
         }
       }
-      float mx0 = -CUDART_INF_F, mx1 = -CUDART_INF_F;
+      // row max: four independent chains of three-input max
+      float m4a = -CUDART_INF_F, m4b = -CUDART_INF_F, m4c = -CUDART_INF_F, m4d = -CUDART_INF_F;
 #pragma unroll
-      for (int c = 0; c < kTile; c += 2) {
-        mx0 = fmaxf(mx0, sv[c]);
-        mx1 = fmaxf(mx1, sv[c + 1]);
+      for (int c = 0; c < kTile; c += 8) {
+        m4a = max3f(m4a, sv[c], sv[c + 1]);
+        m4b = max3f(m4b, sv[c + 2], sv[c + 3]);
+        m4c = max3f(m4c, sv[c + 4], sv[c + 5]);
+        m4d = max3f(m4d, sv[c + 6], sv[c + 7]);
       }
-      const float m_new = fmaxf(m_run, fmaxf(mx0, mx1) * scale_log2);
+      const float m_new = fmaxf(m_run, fmaxf(fmaxf(m4a, m4b), fmaxf(m4c, m4d)) * scale_log2);
       const bool grow = m_new > m_run + kRescaleThreshold || (m_run == -CUDART_INF_F && m_new != -CUDART_INF_F);
       const float m_use = grow ? m_new : m_run;
       const float m_sub = m_use == -CUDART_INF_F ? 0.f : m_use;
       const float alpha = grow ? ex2_approx(m_run - m_use) : 1.f;
-      float rs0 = 0.f, rs1 = 0.f;
-      // exponentials, packed to bf16 pairs in place: u[0..63] holds P's row
+      // exponentials on pairs: x = s * scale - m with one packed FMA; one pair
+      // in kPolyEvery goes through the FMA-pipe polynomial, the rest through
+      // the MUFU, so both units share the load. P is packed to bf16 pairs in
+      // place (u[0..63]); the row sum runs in two packed accumulators.
+      const uint64_t sc2 = f2_pack(scale_log2, scale_log2), nm2 = f2_pack(-m_sub, -m_sub);
+      uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = acc0;
 #pragma unroll
       for (int c = 0; c < kTile; c += 2) {
-        const float e0 = ex2_approx(fmaf(sv[c], scale_log2, -m_sub));
-        const float e1 = ex2_approx(fmaf(sv[c + 1], scale_log2, -m_sub));
-        rs0 += e0;
-        rs1 += e1;
+        float x0, x1;
+        f2_unpack(f2_fma(f2_pack(sv[c], sv[c + 1]), sc2, nm2), x0, x1);
+        uint64_t e;
+        if (((c >> 1) % kPolyEvery) == kPolyEvery - 1)
+          e = f2_exp2_poly(x0, x1);
+        else
+          e = f2_pack(ex2_approx(x0), ex2_approx(x1));
+        if ((c >> 1) & 1)
+          acc1 = f2_add(acc1, e);
+        else
+          acc0 = f2_add(acc0, e);
+        float e0, e1;
+        f2_unpack(e, e0, e1);
         u[c >> 1] = pack_bf16x2(e0, e1);
       }
+      float rs0, rs1;
+      f2_unpack(f2_add(acc0, acc1), rs0, rs1);
       // O may be rescaled once this tile's previous P V has completed; the
       // shared P buffer is free once the other tile's latest P V has
       if (j > 0 && !mbar_wait(&s.o_ready[t], (j - 1) & 1, abort)) {
