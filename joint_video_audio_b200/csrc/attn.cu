@@ -13,20 +13,23 @@
 //               ring of shared-memory slots
 //   warp 1      TMEM allocator + single-thread MMA issuer, in the order
 //                 S0_0 S1_0 | PV0_0 S0_1 PV1_0 S1_1 | PV0_1 S0_2 PV1_1 S1_2 | ...
-//               with Sq_j = Qq K_j^T (M=128, N=128, K=head_dim) and
-//               PVq_j: Oq += Pq_j V_j (M=128, N=head_dim, K=128)
+//               with Sq_j = Qq K_j^T (M=128, N=128, K=head_dim; both operands in
+//               shared memory) and PVq_j: Oq += Pq_j V_j (M=128, N=head_dim,
+//               K=128; P in tensor memory, V in shared memory read MN-major)
 //   warps 2..5  softmax of query tile 0, warps 6..9 of query tile 1; one
 //               thread per query row: S row from TMEM, mask, online max / sum
-//               in the exp2 domain, P (bf16) into shared memory in the
-//               swizzled K-major layout the MMA reads, and the rescale of O in
-//               TMEM when the running max grows by more than 2^8 (otherwise the
-//               stale max is kept, so P stays below 256).
-// The two query tiles share one P buffer: P1_j is written once P0_j V_j has
-// completed and P0_{j+1} once P1_j V_j has, which the MMA order above allows
-// without a bubble (an S product runs in between). That frees shared memory
-// for a four-slot K/V ring, so K_{j+1} and V_{j+1} are fetched one full
-// iteration ahead.
-// Tensor memory: S0 | S1 | O0 | O1 (128 columns each).
+//               in the exp2 domain, P packed to bf16 pairs and stored back
+//               into the first 64 columns of its own S in TMEM, and the rescale
+//               of O in TMEM when the running max grows by more than 2^8
+//               (otherwise the stale max is kept, so P stays below 256).
+// The P V product reads P straight from tensor memory (A operand in TMEM, V
+// from shared memory), so P never touches shared memory: the shared-memory
+// port only feeds Q, K and V, and a five-slot K/V ring fits next to the two
+// query tiles. Ordering needs no extra barriers: the tensor core runs one
+// CTA's MMAs in issue order, so S_t of tile j completing implies P_t V of
+// tile j-1 completed (O_t is stable and P_t's columns are free), and S_t of
+// tile j+1 is issued only after P_t V of tile j.
+// Tensor memory: S0/P0 | S1/P1 | O0 | O1 (128 columns each).
 // KV tiles whose rows all lie in the other document are skipped when neither
 // query tile needs them; tiles that mix documents, run past the end of the
 // sequence, or belong to the other document of one of the two query tiles are
@@ -50,14 +53,13 @@ constexpr int kPolyEvery = 4;  // one exponential pair in four on the FMA pipe
 
 template <int D>
 struct AttnSmem {
-  static constexpr int kSlots = D == 128 ? 4 : 8;
+  static constexpr int kSlots = D == 128 ? 5 : 10;
   static constexpr int kQBytes = kTile * D * 2;     // one query tile
   static constexpr int kKVBytes = kTile * D * 2;    // one K or V tile
-  static constexpr int kPBytes = kTile * kTile * 2; // one P tile
   static constexpr int kRegion = kTile * 128;       // 128 rows x 128 bytes (one swizzle region)
-  static constexpr size_t kBytes = 1024 + 2 * (size_t)kQBytes + (size_t)kPBytes + kSlots * (size_t)kKVBytes + 512;
-  uint8_t *q0, *p, *slot0;  // query tile t at q0 + t * kQBytes, ring slot i at slot0 + i * kKVBytes
-  uint64_t *q_full, *ring_full, *ring_empty, *s_full, *s_free, *p_full, *o_ready, *o_final;
+  static constexpr size_t kBytes = 1024 + 2 * (size_t)kQBytes + kSlots * (size_t)kKVBytes + 512;
+  uint8_t *q0, *slot0;  // query tile t at q0 + t * kQBytes, ring slot i at slot0 + i * kKVBytes
+  uint64_t *q_full, *ring_full, *ring_empty, *s_full, *p_full, *o_final;
   uint32_t* tmem_base;
   int* abort;
 
@@ -66,8 +68,6 @@ struct AttnSmem {
     uint8_t* x = raw + (((base + 1023u) & ~1023u) - base);
     q0 = x;
     x += 2 * kQBytes;
-    p = x;
-    x += kPBytes;
     slot0 = x;
     x += kSlots * kKVBytes;
     uint64_t* b = reinterpret_cast<uint64_t*>(x);
@@ -75,12 +75,10 @@ struct AttnSmem {
     ring_full = b + 1;
     ring_empty = b + 1 + kSlots;
     s_full = b + 1 + 2 * kSlots;
-    s_free = s_full + 2;
-    p_full = s_full + 4;
-    o_ready = s_full + 6;
-    o_final = s_full + 8;
-    tmem_base = reinterpret_cast<uint32_t*>(s_full + 9);
-    abort = reinterpret_cast<int*>(s_full + 10);
+    p_full = s_full + 2;
+    o_final = s_full + 4;
+    tmem_base = reinterpret_cast<uint32_t*>(s_full + 5);
+    abort = reinterpret_cast<int*>(s_full + 6);
   }
 };
 
@@ -140,9 +138,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s.s_full[i], 1);
-      mbar_init(&s.s_free[i], 4);
       mbar_init(&s.p_full[i], 4);
-      mbar_init(&s.o_ready[i], 1);
     }
     mbar_init(s.o_final, 1);
     *s.abort = 0;
@@ -204,7 +200,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       auto wait_ring = [&](int u) { return mbar_wait(&s.ring_full[u % kSlots], (u / kSlots) & 1, abort); };
       // S_t = Q_t K_j^T into TMEM columns [t*128, t*128+128)
       auto issue_s = [&](int t, int j) -> bool {
-        if (j > 0 && !mbar_wait(&s.s_free[t], (j - 1) & 1, abort)) return false;
         tc_fence_after();
         const uint32_t qa = q0 + t * SM::kQBytes;
         const uint32_t ka = ring0 + slot_of(2 * j) * SM::kKVBytes;
@@ -217,19 +212,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         mma_commit(&s.s_full[t]);
         return true;
       };
-      // O_t += P_t V_j into TMEM columns [256 + t*128, ...)
+      // O_t += P_t V_j into TMEM columns [256 + t*128, ...); P_t is read from
+      // TMEM columns [t*128, t*128 + 64), 8 columns per K = 16 step
       auto issue_pv = [&](int t, int j) -> bool {
         if (!mbar_wait(&s.p_full[t], j & 1, abort)) return false;
         tc_fence_after();
-        const uint32_t pa = smem_u32(s.p);
         const uint32_t va = ring0 + slot_of(2 * j + 1) * SM::kKVBytes;
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk) {
-          const uint64_t ad = sw128_desc(pa + (kk >> 2) * SM::kRegion + (kk & 3) * 32, 16);
           const uint64_t bd = sw128_desc(va + kk * 16 * 128, SM::kRegion);
-          mma_bf16_ss(tmem + 256 + t * kTile, ad, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_bf16_ts(tmem + 256 + t * kTile, tmem + t * kTile + kk * 8, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
         }
-        mma_commit(&s.o_ready[t]);
         return true;
       };
       bool ok = mbar_wait(s.q_full, 0, abort);
@@ -271,7 +264,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     const float scale_log2 = 1.4426950408889634f * rsqrtf((float)D);
     const int myk = t == 0 ? qk0 : qk1;
     float m_run = -CUDART_INF_F, l_run = 0.f;
-    uint8_t* prow = s.p + r * 128;
     bool ok = true;
     int j = 0;
     for (int kt = next_kv_tile(p.tiles, n_tiles, qk0, qk1, 0); kt < n_tiles;
@@ -283,9 +275,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       tc_fence_after();
       uint32_t u[kTile];
       tmem_ld128(t_s, u);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s.s_free[t]);
       float* sv = reinterpret_cast<float*>(u);
       {
         const TileInfo& ti = p.tiles[kt];
@@ -322,35 +311,29 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       const uint64_t sc2 = f2_pack(scale_log2, scale_log2), nm2 = f2_pack(-m_sub, -m_sub);
       uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = acc0;
 #pragma unroll
-      for (int c = 0; c < kTile; c += 2) {
-        float x0, x1;
-        f2_unpack(f2_fma(f2_pack(sv[c], sv[c + 1]), sc2, nm2), x0, x1);
-        uint64_t e;
-        if (((c >> 1) % kPolyEvery) == kPolyEvery - 1)
-          e = f2_exp2_poly(x0, x1);
-        else
-          e = f2_pack(ex2_approx(x0), ex2_approx(x1));
-        if ((c >> 1) & 1)
-          acc1 = f2_add(acc1, e);
-        else
-          acc0 = f2_add(acc0, e);
-        float e0, e1;
-        f2_unpack(e, e0, e1);
-        u[c >> 1] = pack_bf16x2(e0, e1);
+      for (int h = 0; h < 2; ++h) {  // two halves of 64 columns -> 32 packed words each
+#pragma unroll
+        for (int c = 64 * h; c < 64 * h + 64; c += 2) {
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(sv[c], sv[c + 1]), sc2, nm2), x0, x1);
+          uint64_t e;
+          if (((c >> 1) % kPolyEvery) == kPolyEvery - 1)
+            e = f2_exp2_poly(x0, x1);
+          else
+            e = f2_pack(ex2_approx(x0), ex2_approx(x1));
+          if ((c >> 1) & 1)
+            acc1 = f2_add(acc1, e);
+          else
+            acc0 = f2_add(acc0, e);
+          float e0, e1;
+          f2_unpack(e, e0, e1);
+          u[c >> 1] = pack_bf16x2(e0, e1);
+        }
+        // P half -> tensor memory, over the first 64 columns of this tile's S
+        tmem_st32(t_s + 32 * h, *reinterpret_cast<const uint32_t(*)[32]>(u + 32 * h));
       }
       float rs0, rs1;
       f2_unpack(f2_add(acc0, acc1), rs0, rs1);
-      // O may be rescaled once this tile's previous P V has completed; the
-      // shared P buffer is free once the other tile's latest P V has
-      if (j > 0 && !mbar_wait(&s.o_ready[t], (j - 1) & 1, abort)) {
-        ok = false;
-        break;
-      }
-      if (t == 0 ? (j > 0 && !mbar_wait(&s.o_ready[1], (j - 1) & 1, abort))
-                 : !mbar_wait(&s.o_ready[0], j & 1, abort)) {
-        ok = false;
-        break;
-      }
       if (j > 0 && __any_sync(0xffffffffu, grow)) {
         tc_fence_after();
 #pragma unroll 1
@@ -365,14 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       }
       l_run = l_run * alpha + (rs0 + rs1);
       m_run = m_use;
-      // P row -> shared memory, 128-byte swizzle, two 64-column regions
-#pragma unroll
-      for (int c = 0; c < kTile / 8; ++c) {
-        const int region = c >> 3, cc = c & 7;
-        *reinterpret_cast<uint4*>(prow + region * SM::kRegion + ((cc ^ (r & 7)) << 4)) =
-            make_uint4(u[4 * c], u[4 * c + 1], u[4 * c + 2], u[4 * c + 3]);
-      }
-      fence_proxy_async_smem();
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s.p_full[t]);
