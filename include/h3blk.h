@@ -217,6 +217,26 @@ H3BLK_API int h3blk_gemm_s8_s32(int64_t M, int N, int K, const int8_t* A, const 
  * (K a multiple of 64, N a multiple of 128). */
 H3BLK_API int h3blk_gemm_bf16(int64_t M, int N, int K, const void* A, const void* B, void* C, void* stream);
 
+/* Document-masked attention of the block (the same kernels as the attention
+ * step of h3blk_forward) for callers that cannot allocate device memory at run
+ * time, such as a plugin inside a host application whose memory pool owns the
+ * GPU's memory, or a latency-critical loop that cannot afford the device-wide
+ * synchronisation of cudaMalloc / cudaFree. It needs no workspace: its scratch
+ * (tile summary and error word) is a fixed ~128 KiB array in the library's
+ * own device memory, held by every GPU that loads the library until exit.
+ * The pages have no counterpart of this entry point.
+ *   qkv  bf16 [N, 3*heads*head_dim]  (the layout of H3BLK_STAGE_QKV)
+ *   tag, tidx int32 [N]              (as for h3blk_forward; tidx only validated)
+ *   o    bf16 [N, heads*head_dim]    output
+ * UNSUPPORTED when n_rows > 524,288 (the fixed scratch's limit) or head_dim is
+ * not 64 / 128. It calls no allocator. All calls share the one scratch array,
+ * which keeps the last call's contents: calls that overlap on the GPU race,
+ * so serialise them. The first call on each device looks up the array's
+ * device address; make that first call before any stream capture. */
+H3BLK_API int h3blk_attention_noalloc(int64_t n_rows, int heads, int head_dim, int n_tags, int n_t,
+                                      const void* qkv, const int32_t* tag, const int32_t* tidx, void* o,
+                                      void* stream);
+
 /* Message for a status code (static storage). */
 H3BLK_API const char* h3blk_error_string(int status);
 

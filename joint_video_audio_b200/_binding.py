@@ -27,7 +27,7 @@ STAGE = {name: i for i, name in enumerate(STAGES)}
 EXPORTS = ["h3blk_create", "h3blk_destroy", "h3blk_workspace_bytes", "h3blk_stage_view", "h3blk_forward",
            "h3blk_check", "h3blk_int8_weights_bytes", "h3blk_prepare_int8_weights", "h3blk_rotate_quantize",
            "h3blk_gemm_s8_s32", "h3blk_gemm_bf16", "h3blk_error_string", "h3blk_version",
-           "h3blk_set_kernel_events"]
+           "h3blk_set_kernel_events", "h3blk_attention_noalloc"]
 
 H3BLK_TIMING_POINTS = 11
 TIMING_INTERVALS = ["prep", "norm1", "qkv_gemm", "attention", "quant_o", "out_proj_gemm", "norm2",
@@ -73,6 +73,7 @@ def _load():
         "h3blk_error_string": (C.c_char_p, [i32]),
         "h3blk_version": (i32, []),
         "h3blk_set_kernel_events": (i32, [vp, C.POINTER(vp), i32]),
+        "h3blk_attention_noalloc": (i32, [i64, i32, i32, i32, i32, vp, vp, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -180,3 +181,9 @@ def h3blk_set_kernel_events(handle, events) -> None:
         return
     arr = (C.c_void_p * len(events))(*events)
     _check("h3blk_set_kernel_events", _lib.h3blk_set_kernel_events(handle, arr, len(events)))
+
+
+def h3blk_attention_noalloc(n_rows, heads, head_dim, n_tags, n_t, qkv, tag, tidx, o, stream) -> int:
+    """Raw call (pointers are ints); returns the status code. Uses the
+    library's fixed device scratch instead of a caller workspace."""
+    return _lib.h3blk_attention_noalloc(n_rows, heads, head_dim, n_tags, n_t, qkv, tag, tidx, o, stream)
