@@ -1,0 +1,158 @@
+"""GPU parity at the real dimensions and full sequence lengths, in the launch
+configuration bench.py times (one h3blk_forward per sequence).
+
+real_8k is compared end to end against the fp64 oracle (k and v for all 8192
+rows, every other stage on 256 seeded rows). The larger sequences (32k, 32k
+with padding, the 54k ref2va layout, the W8A8 32k layout) are checked stage by
+stage on 256 seeded rows plus 8 padding rows: each stage is recomputed by the
+oracle from the GPU's own input to that stage (attention from the GPU's q of
+the sampled rows and the GPU's k, v of every row), so each kernel is checked
+at full size without an fp64 pass over the whole sequence. Padding rows are
+checked on all rows: out == x bit for bit.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import h3_inputs as hi
+from oracle import h3_block as orc
+from tests._parity import GpuCase, assert_intermediate, assert_stage, to64
+
+pytestmark = pytest.mark.gpu
+
+
+def _rows_gpu(t, rows):
+    return t[torch.as_tensor(rows, device=t.device)]
+
+
+def _stage_chain(case: GpuCase, ob: orc.BlockOracle, rows):
+    """Each stage of the sampled rows against the oracle fed with the GPU's
+    own input to that stage."""
+    d = case.dims
+    lay = case.inp.layout
+    hd = d.heads * d.head_dim
+    table = orc.f64(case.inp.table)
+    x = orc.f64(case.inp.x[torch.as_tensor(rows)])
+    m = orc.modulation(table, lay.tag[rows], lay.tidx[rows])
+    quant = bool(d.quant)
+
+    # pre-attention norm (from the inputs)
+    h1 = orc.adaln(x, m[:, orc.MOD_SHIFT1], m[:, orc.MOD_SCALE1], d.norm_eps)
+    if quant:
+        q8 = _rows_gpu(case.stage("H1_Q8"), rows).cpu().numpy()
+        rq, _ = orc.quantize_rows(orc.rotate_blocks(h1))
+        dq = np.abs(q8.astype(np.int64) - rq.astype(np.int64))
+        assert dq.max() <= 1 and np.mean(dq == 0) >= 0.999
+    else:
+        h1_g = _rows_gpu(case.stage("H1"), rows)
+        assert_intermediate("h1", h1_g, h1)
+
+    # QKV GEMM + QK-norm + RoPE, from the GPU's h1 (or its int8 operand)
+    if quant:
+        q8 = _rows_gpu(case.stage("H1_Q8"), rows).cpu().numpy()
+        s8 = _rows_gpu(case.stage("H1_SCALE"), rows).cpu().numpy().astype(np.float64)
+        wq, sw = ob.int8["qkv"]
+        y = orc.int8_matmul_exact(q8, wq).astype(np.float64) * s8[:, None] * sw[None, :]
+    else:
+        y = orc.f64(h1_g) @ ob.wqkv.T
+    sh = lambda a: a.reshape(len(rows), d.heads, d.head_dim)  # noqa: E731
+    pos = lay.pos[rows]
+    q_ref = orc.apply_rope(orc.qk_rmsnorm(sh(y[:, :hd]), ob.q_gain, d.qk_norm_eps), pos, d.rope_pairs, d.rope_theta)
+    k_ref = orc.apply_rope(orc.qk_rmsnorm(sh(y[:, hd:2 * hd]), ob.k_gain, d.qk_norm_eps), pos, d.rope_pairs, d.rope_theta)
+    qg, kg, vg = case.qkv(rows)
+    assert_intermediate("q", qg, q_ref)
+    assert_intermediate("k", kg, k_ref)
+    assert_intermediate("v", vg, sh(y[:, 2 * hd:]))
+
+    # attention of the sampled queries over the GPU's k, v of every row
+    # (queries in chunks to bound host memory)
+    qkv_all = case.stage("QKV")
+    k_all = qkv_all[:, hd:2 * hd].float().cpu().numpy().reshape(-1, d.heads, d.head_dim)
+    v_all = qkv_all[:, 2 * hd:].float().cpu().numpy().reshape(-1, d.heads, d.head_dim)
+    doc = orc.documents(lay.tag)
+    qn = to64(qg)
+    o_ref = np.concatenate([orc.attention(qn[i:i + 32], k_all, v_all, doc[rows[i:i + 32]], doc)
+                            for i in range(0, len(rows), 32)]).reshape(len(rows), hd)
+    del k_all, v_all
+    o_g = _rows_gpu(case.stage("O"), rows)
+    assert_intermediate("o", o_g, o_ref)
+
+    # out-projection + gated residual, from the GPU's o
+    if quant:
+        oq = _rows_gpu(case.stage("O_Q8"), rows).cpu().numpy()
+        os_ = _rows_gpu(case.stage("O_SCALE"), rows).cpu().numpy().astype(np.float64)
+        rq, _ = orc.quantize_rows(orc.rotate_blocks(to64(o_g)))
+        dq = np.abs(oq.astype(np.int64) - rq.astype(np.int64))
+        assert dq.max() <= 1 and np.mean(dq == 0) >= 0.999
+        wq, sw = ob.int8["o"]
+        yo = orc.int8_matmul_exact(oq, wq).astype(np.float64) * os_[:, None] * sw[None, :]
+    else:
+        yo = to64(o_g) @ ob.wo.T
+    x1_g = _rows_gpu(case.stage("X1"), rows)
+    assert_intermediate("x1", x1_g, x + m[:, orc.MOD_GATE1] * yo)
+
+    # pre-FFN norm, FFN up + SwiGLU, from the GPU's x1
+    h2 = orc.adaln(to64(x1_g), m[:, orc.MOD_SHIFT2], m[:, orc.MOD_SCALE2], d.norm_eps)
+    if quant:
+        h2q = _rows_gpu(case.stage("H2_Q8"), rows).cpu().numpy()
+        h2s = _rows_gpu(case.stage("H2_SCALE"), rows).cpu().numpy().astype(np.float64)
+        rq, _ = orc.quantize_rows(orc.rotate_blocks(h2))
+        dq = np.abs(h2q.astype(np.int64) - rq.astype(np.int64))
+        assert dq.max() <= 1 and np.mean(dq == 0) >= 0.999
+        wq, sw = ob.int8["13"]
+        gu = orc.int8_matmul_exact(h2q, wq).astype(np.float64) * h2s[:, None] * sw[None, :]
+    else:
+        h2_g = _rows_gpu(case.stage("H2"), rows)
+        assert_intermediate("h2", h2_g, h2)
+        gu = to64(h2_g) @ ob.w13.T
+    a_g = _rows_gpu(case.stage("A"), rows)
+    assert_intermediate("a", a_g, orc.swiglu(gu[:, :d.ffn], gu[:, d.ffn:]))
+
+    # FFN down + gated residual, from the GPU's a
+    if quant:
+        aq = _rows_gpu(case.stage("A_Q8"), rows).cpu().numpy()
+        as_ = _rows_gpu(case.stage("A_SCALE"), rows).cpu().numpy().astype(np.float64)
+        wq, sw = ob.int8["2"]
+        yd = orc.int8_matmul_exact(aq, wq).astype(np.float64) * as_[:, None] * sw[None, :]
+    else:
+        yd = to64(a_g) @ ob.w2.T
+    out_g = _rows_gpu(case.out, rows)
+    assert_stage("out", out_g, to64(x1_g) + m[:, orc.MOD_GATE2] * yd)
+
+
+def _check_padding(case: GpuCase):
+    pad = torch.from_numpy(case.inp.layout.tag == -1).cuda()
+    if bool(pad.any()):
+        assert torch.equal(case.out[pad], case.x[pad])
+
+
+@pytest.mark.parametrize("name", ["t2va_32k", "t2va_32k_pad168", "ref2va_54k", "w8a8_t2va_32k"])
+def test_fullsize_stage_chain(name):
+    dims, lay = hi.workload(name)
+    inp = hi.make_inputs(dims, lay)
+    case = GpuCase(inp)
+    case.run()
+    assert case.block.check(case.ws, case.n) == 0
+    _check_padding(case)
+    ob = orc.BlockOracle(dims, inp.weights)
+    rows = hi.sample_rows(lay, k=256, k_pad=8)
+    _stage_chain(case, ob, rows)
+
+
+def test_real_8k_end_to_end_vs_oracle():
+    dims, lay = hi.workload("real_8k")
+    inp = hi.make_inputs(dims, lay)
+    case = GpuCase(inp)
+    case.run()
+    rows = hi.sample_rows(lay, k=256, k_pad=8)
+    ref = orc.BlockOracle(dims, inp.weights).forward(inp.x, lay.tag, lay.tidx, lay.pos, inp.table, rows=rows)
+    assert_intermediate("h1", _rows_gpu(case.stage("H1"), rows), ref["h1"])
+    qg, kg, vg = case.qkv(rows)
+    assert_intermediate("q", qg, ref["q"])
+    assert_intermediate("k", kg, ref["k"])
+    assert_intermediate("v", vg, ref["v"])
+    assert_intermediate("o", _rows_gpu(case.stage("O"), rows), ref["o"])
+    assert_intermediate("x1", _rows_gpu(case.stage("X1"), rows), ref["x1"])
+    assert_intermediate("a", _rows_gpu(case.stage("A"), rows), ref["a"])
+    assert_stage("out", _rows_gpu(case.out, rows), ref["out"])
