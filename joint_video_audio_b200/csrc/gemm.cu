@@ -3,8 +3,9 @@
 //
 //   warp 0      TMA producer: A tile 128 x 128 B and B tile 256 x 128 B per stage
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
-//   warps 2..5  epilogue: tcgen05.ld of the fp32 / s32 accumulator (thread =
-//               output row), fused math, 16-byte global stores
+//   warps 2..9  epilogue: tcgen05.ld of the fp32 / s32 accumulator (thread =
+//               output row; the two warps of a lane quadrant take one half of
+//               the tile's columns each), fused math, 16-byte global stores
 //
 // Accumulators are double-buffered in tensor memory (2 x 256 columns) so the
 // epilogue of tile i overlaps the main loop of tile i+1. Operands are staged by
@@ -36,7 +37,8 @@ constexpr int kRowBytes = 128;  // one K-block per stage: 64 bf16 or 128 int8
 constexpr int kStages = 4;
 constexpr int kAStage = BM * kRowBytes;  // 16 KB
 constexpr int kBStage = BN * kRowBytes;  // 32 KB
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;  // two per TMEM lane quadrant, each on one half of the tile's columns
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kTmemCols = 512;  // two 256-column fp32 accumulators
 constexpr int kGroupN = 8;      // tile raster: 8 N-tiles share each pass over M
 constexpr size_t kSmemBytes = 1024 + (size_t)kStages * (kAStage + kBStage) + 256;
@@ -118,12 +120,13 @@ __device__ __forceinline__ void load_chunk(uint32_t taddr, float sa, const float
 
 // ------------------------------------------------------------------ epilogue
 template <int EPI, bool INT8>
-__device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tacc, int64_t row, bool row_ok, int n_tile) {
+__device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tacc, int64_t row, bool row_ok, int n_tile,
+                                              int half) {
   const float sa = (INT8 && row_ok) ? __ldg(p.s_a + row) : 0.f;
   if (EPI == kEpiSwiGLU) {
     const int col0 = n_tile * 128;
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 2 * half; c < 2 * half + 2; ++c) {
       float g[32], u[32];
       load_chunk<INT8>(tacc + c * 32, sa, p.s_b, col0 + c * 32, g);
       load_chunk<INT8>(tacc + 128 + c * 32, sa, p.s_b, p.N + col0 + c * 32, u);
@@ -134,9 +137,10 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tacc, 
     return;
   }
   const int n0 = n_tile * BN;
+  constexpr int kHalfChunks = BN / 64;  // 32-column chunks in one half of the tile
   if (EPI == kEpiStoreS32) {
 #pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
+    for (int c = half * kHalfChunks; c < (half + 1) * kHalfChunks; ++c) {
       if (n0 + c * 32 >= p.N) break;
       uint32_t r[32];
       tmem_ld32(tacc + c * 32, r);
@@ -156,7 +160,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tacc, 
         gate = p.table + (((int64_t)tg * p.n_t + ti) * 6 + p.gate_idx) * p.N;
     }
 #pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
+    for (int c = half * kHalfChunks; c < (half + 1) * kHalfChunks; ++c) {
       const int col = n0 + c * 32;
       if (col >= p.N) break;
       float v[32];
@@ -196,8 +200,9 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tacc, 
       pos3[1] = __ldg(p.pos + row * 3 + 1);
       pos3[2] = __ldg(p.pos + row * 3 + 2);
     }
+    const int heads_per_half = (BN / 2) / D;
 #pragma unroll 1
-    for (int hh = 0; hh < BN / D; ++hh) {
+    for (int hh = half * heads_per_half; hh < (half + 1) * heads_per_half; ++hh) {
       const int col0 = n0 + hh * D;
       if (col0 >= p.N) break;
       const int region = col0 / p.hd;  // 0 q, 1 k, 2 v
@@ -267,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s.tfull[i], 1);
-      mbar_init(&s.tempty[i], 4);  // one arrival per epilogue warp
+      mbar_init(&s.tempty[i], kEpiWarps);  // one arrival per epilogue warp
     }
     mbar_init(s.drain, 1);
     *s.abort = 0;
@@ -385,6 +390,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ---------------------------------------------------------------- epilogue
     const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;
     int local = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++local) {
       const TileCoord tc = tile_coord(t, tiles_m, tiles_n);
@@ -397,7 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const int64_t row = (int64_t)tc.m * BM + quad * 32 + lane;
       const uint32_t tacc = tmem_base + ((uint32_t)(quad * 32) << 16) + buf * BN;
-      epilogue_tile<EPI, INT8>(p, tacc, row, row < p.M, tc.n);
+      epilogue_tile<EPI, INT8>(p, tacc, row, row < p.M, tc.n, half);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s.tempty[buf]);
@@ -441,7 +447,7 @@ cudaError_t launch_gemm(const GemmArgs& a, PFN_cuTensorMapEncodeTiled_v12000 enc
   if (a.M <= 0) return cudaSuccess;
   const int kb = a.int8 ? 128 : 64;
   if (a.K % kb != 0 || a.N % 128 != 0 || a.Nb % 128 != 0) return cudaErrorInvalidValue;
-  if (a.epi == kEpiQKV && (a.head_dim % 32 != 0 || BN % a.head_dim != 0 || a.hd % a.head_dim != 0))
+  if (a.epi == kEpiQKV && (a.head_dim % 32 != 0 || (BN / 2) % a.head_dim != 0 || a.hd % a.head_dim != 0))
     return cudaErrorInvalidValue;
   CUtensorMap ta, tb;
   if (make_map(encode, &ta, a.A, (uint64_t)a.M, (uint64_t)a.K, a.int8) != CUDA_SUCCESS) return cudaErrorInvalidValue;
