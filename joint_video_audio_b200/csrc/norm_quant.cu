@@ -151,11 +151,10 @@ __global__ void __launch_bounds__(256) modnorm_bf16_kernel(ModNormArgs a) {
 }
 
 // ============================================================== rotation + quant
-// One CTA of 256 threads per row; thread t owns chunks t, t+256, ... of 8
-// channels. A 128-channel Hadamard block is 16 consecutive chunks, i.e. one
-// half-warp, so the transform is 3 in-register butterfly stages followed by
-// 4 shuffle stages.
-constexpr int kRQThreads = 256;
+// One CTA per row at a time; thread t owns chunks t, t + THREADS, ... of 8
+// channels (THREADS a multiple of 16). A 128-channel Hadamard block is 16
+// consecutive chunks, i.e. one half-warp, so the transform is 3 in-register
+// butterfly stages followed by 4 shuffle stages.
 
 __device__ __forceinline__ void fwht128_chunk(float (&h)[8], int lane) {
 #pragma unroll
@@ -210,83 +209,106 @@ __device__ __forceinline__ void quant_store(const float (&h)[8], float s, bool z
 }
 
 // MODNORM = true: the row is x, modulated and normalised first (K1 fused).
-template <int CPT, bool MODNORM>
-__global__ void __launch_bounds__(kRQThreads) rotate_quant_kernel(const __nv_bfloat16* __restrict__ in, int K,
-                                                                  int8_t* __restrict__ out_q,
-                                                                  float* __restrict__ out_scale, ModNormArgs a) {
-  __shared__ float red[kRQThreads / 32];
-  const int64_t row = blockIdx.x;
+// One CTA per row.
+template <int CPT, int THREADS, bool MODNORM>
+__global__ void __launch_bounds__(THREADS) rotate_quant_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows,
+                                                               int K, int8_t* __restrict__ out_q,
+                                                               float* __restrict__ out_scale, ModNormArgs a) {
+  __shared__ float red[THREADS / 32];
   const int lane = threadIdx.x & 31;
   const int nchunk = K >> 3;
-  const uint4* src = reinterpret_cast<const uint4*>(in + row * (int64_t)K);
-  float h[CPT][8];
-  float ss = 0.f;
-#pragma unroll
-  for (int i = 0; i < CPT; ++i) {
-    const int c = threadIdx.x + kRQThreads * i;
-    if (c < nchunk) {
-      bf16x8_to_f32(ld_nc_v4(src + c), h[i]);
-    } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) h[i][e] = 0.f;
-    }
-    if (MODNORM) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) ss = fmaf(h[i][e], h[i][e], ss);
-    }
-  }
-  if (MODNORM) {
-    ss = block_reduce(ss, false, red);
-    const float rstd = rsqrtf(ss / (float)K + a.eps);
-    const float* m = mod_row(a.table, a.tag, a.tidx, row, a.n_tags, a.n_t, K);
+  const int64_t row = blockIdx.x;
+  if (row >= rows) return;
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(in + row * (int64_t)K);
+    float h[CPT][8];
 #pragma unroll
     for (int i = 0; i < CPT; ++i) {
-      const int c = threadIdx.x + kRQThreads * i;
+      const int c = threadIdx.x + THREADS * i;
       if (c < nchunk) {
+        bf16x8_to_f32(ld_nc_v4(src + c), h[i]);
+      } else {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float sh = m ? __ldg(m + (int64_t)a.shift_idx * K + c * 8 + e) : 0.f;
-          const float sc = m ? __ldg(m + (int64_t)a.scale_idx * K + c * 8 + e) : 0.f;
-          h[i][e] = fmaf(h[i][e] * rstd, 1.f + sc, sh);
-        }
+        for (int e = 0; e < 8; ++e) h[i][e] = 0.f;
       }
     }
-  }
-  float amax = 0.f;
+    if (MODNORM) {
+      float ss = 0.f;
 #pragma unroll
-  for (int i = 0; i < CPT; ++i) {
-    // all 32 lanes take part in the shuffles; out-of-range chunks hold zeros
-    fwht128_chunk(h[i], lane);
+      for (int i = 0; i < CPT; ++i)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(h[i][e]));
-  }
-  amax = block_reduce(amax, true, red);
-  const float s = amax / 127.f;
-  const bool zero = !(amax > 0.f);
-  if (threadIdx.x == 0) out_scale[row] = s;
-  int8_t* dst = out_q + row * (int64_t)K;
+        for (int e = 0; e < 8; ++e) ss = fmaf(h[i][e], h[i][e], ss);
+      ss = block_reduce(ss, false, red);
+      const float rstd = rsqrtf(ss / (float)K + a.eps);
+      const float* m = mod_row(a.table, a.tag, a.tidx, row, a.n_tags, a.n_t, K);
 #pragma unroll
-  for (int i = 0; i < CPT; ++i) {
-    const int c = threadIdx.x + kRQThreads * i;
-    if (c < nchunk) quant_store(h[i], s, zero, dst + c * 8);
+      for (int i = 0; i < CPT; ++i) {
+        const int c = threadIdx.x + THREADS * i;
+        float sh[8], sc[8];
+        if (m && c < nchunk) {
+          const float4* s4 = reinterpret_cast<const float4*>(m + (int64_t)a.shift_idx * K + c * 8);
+          const float4* k4 = reinterpret_cast<const float4*>(m + (int64_t)a.scale_idx * K + c * 8);
+          const float4 s0 = __ldg(s4), s1 = __ldg(s4 + 1), k0 = __ldg(k4), k1 = __ldg(k4 + 1);
+          sh[0] = s0.x; sh[1] = s0.y; sh[2] = s0.z; sh[3] = s0.w; sh[4] = s1.x; sh[5] = s1.y; sh[6] = s1.z; sh[7] = s1.w;
+          sc[0] = k0.x; sc[1] = k0.y; sc[2] = k0.z; sc[3] = k0.w; sc[4] = k1.x; sc[5] = k1.y; sc[6] = k1.z; sc[7] = k1.w;
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) sh[e] = sc[e] = 0.f;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) h[i][e] = fmaf(h[i][e] * rstd, 1.f + sc[e], sh[e]);
+      }
+    }
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < CPT; ++i) {
+      // all 32 lanes take part in the shuffles; out-of-range chunks hold zeros
+      fwht128_chunk(h[i], lane);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(h[i][e]));
+    }
+    amax = block_reduce(amax, true, red);
+    const float s = amax / 127.f;
+    const bool zero = !(amax > 0.f);
+    if (threadIdx.x == 0) out_scale[row] = s;
+    int8_t* dst = out_q + row * (int64_t)K;
+#pragma unroll
+    for (int i = 0; i < CPT; ++i) {
+      const int c = threadIdx.x + THREADS * i;
+      if (c < nchunk) quant_store(h[i], s, zero, dst + c * 8);
+    }
   }
 }
 
+template <int CPT, int THREADS, bool MODNORM>
+static cudaError_t launch_rq_t(const __nv_bfloat16* in, int64_t rows, int K, int8_t* q, float* sc,
+                               const ModNormArgs& a, cudaStream_t s) {
+  // one CTA per row (measured faster here than a persistent grid that
+  // prefetches the next row)
+  rotate_quant_kernel<CPT, THREADS, MODNORM><<<(unsigned)rows, THREADS, 0, s>>>(in, rows, K, q, sc, a);
+  return cudaGetLastError();
+}
+
+// Thread count and chunks per thread for a row of K channels: exact fits for
+// the block's widths, otherwise 256 threads with enough chunks each.
 template <bool MODNORM>
 static cudaError_t launch_rq(const __nv_bfloat16* in, int64_t rows, int K, int8_t* q, float* sc,
                              const ModNormArgs& a, cudaStream_t s) {
-  const int cpt = (K / 8 + kRQThreads - 1) / kRQThreads;
-  const dim3 grid((unsigned)rows), block(kRQThreads);
-  switch (cpt) {
+  const int nchunk = K / 8;
+  if (nchunk == 672) return launch_rq_t<3, 224, MODNORM>(in, rows, K, q, sc, a, s);   // 5376 channels
+  if (nchunk == 896) return launch_rq_t<4, 224, MODNORM>(in, rows, K, q, sc, a, s);   // 7168
+  if (nchunk == 1792) return launch_rq_t<7, 256, MODNORM>(in, rows, K, q, sc, a, s);  // 14336
+  if (nchunk <= 32) return launch_rq_t<1, 32, MODNORM>(in, rows, K, q, sc, a, s);
+  if (nchunk <= 128) return launch_rq_t<1, 128, MODNORM>(in, rows, K, q, sc, a, s);
+  switch ((nchunk + 255) / 256) {
 #define H3_RQ_CASE(N) \
-  case N: rotate_quant_kernel<N, MODNORM><<<grid, block, 0, s>>>(in, K, q, sc, a); break;
+  case N: return launch_rq_t<N, 256, MODNORM>(in, rows, K, q, sc, a, s);
     H3_RQ_CASE(1) H3_RQ_CASE(2) H3_RQ_CASE(3) H3_RQ_CASE(4) H3_RQ_CASE(5) H3_RQ_CASE(6) H3_RQ_CASE(7)
     H3_RQ_CASE(8)
 #undef H3_RQ_CASE
     default:
       return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 cudaError_t launch_rotate_quant(const __nv_bfloat16* in, int64_t rows, int K, int8_t* out_q, float* out_scale,
