@@ -172,7 +172,8 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[3]) if v.lower() == "active"})
         return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in rows),
-                "reasons": reasons, "samples": len(loaded)}
+                "reasons": reasons, "samples": len(loaded),
+                "power_w_median": statistics.median(r[2] for r in loaded), "power_w_max": max(r[2] for r in loaded)}
 
 
 def attention_flops(dims, layout):

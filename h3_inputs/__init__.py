@@ -330,3 +330,59 @@ def sample_rows(layout: Layout, k=256, k_pad=8, seed=0) -> np.ndarray:
     if pad.size:
         rows = np.concatenate([rows, rng.choice(pad, size=min(k_pad, pad.size), replace=False)])
     return np.sort(rows).astype(np.int64)
+
+
+# --------------------------------------------------------------------------
+# Modulation-table producer (timestep embedding -> time MLP -> per-tag AdaLN)
+# --------------------------------------------------------------------------
+
+@dataclass(frozen=True)
+class ModDims:
+    """Timestep embedding / MLP sizes ("MiniMaxH3Transformer3DModel",
+    constructor: freq_dim, time_embed_hidden_dim, time_embed_dim)."""
+    freq_dim: int = 256
+    time_hidden: int = 5376
+    time_dim: int = 2688
+
+
+REAL_MOD = ModDims()
+TINY_MOD = ModDims(freq_dim=64, time_hidden=128, time_dim=64)
+
+
+@dataclass
+class ModParams:
+    md: ModDims
+    w1: torch.Tensor      # fp32 [time_hidden, freq_dim]
+    b1: torch.Tensor      # fp32 [time_hidden]
+    w2: torch.Tensor      # fp32 [time_dim, time_hidden]
+    b2: torch.Tensor      # fp32 [time_dim]
+    w1_r: torch.Tensor | None   # second-time copy (two-time conditioning)
+    b1_r: torch.Tensor | None
+    w2_r: torch.Tensor | None
+    b2_r: torch.Tensor | None
+    adaln_w: torch.Tensor  # bf16 [n_tags, 6C, time_dim]
+    adaln_b: torch.Tensor  # fp32 [n_tags, 6C]
+
+
+def make_modulation_params(dims: Dims, md: ModDims, seed=0, two_time=False) -> ModParams:
+    rng = np.random.default_rng(seed + 50)
+    f = lambda a: torch.from_numpy(a)  # noqa: E731
+
+    def mlp():
+        return (f(_normal(rng, (md.time_hidden, md.freq_dim), 1.0 / np.sqrt(md.freq_dim))),
+                f(_normal(rng, (md.time_hidden,), 0.02)),
+                f(_normal(rng, (md.time_dim, md.time_hidden), 1.0 / np.sqrt(md.time_hidden))),
+                f(_normal(rng, (md.time_dim,), 0.02)))
+    w1, b1, w2, b2 = mlp()
+    r = mlp() if two_time else (None, None, None, None)
+    aw = to_bf16(_normal(rng, (dims.n_tags, 6 * dims.hidden, md.time_dim), 0.1 / np.sqrt(md.time_dim)))
+    ab = f(_normal(rng, (dims.n_tags, 6 * dims.hidden), 0.02))
+    return ModParams(md, w1, b1, w2, b2, *r, aw, ab)
+
+
+def two_time_sets(t_now, t_end):
+    """Per-set timesteps for the two-time table index 2 * i + j: set (i, j)
+    pairs t_now[i] with t_end[j]."""
+    tn = [t_now[i] for i in range(len(t_now)) for _ in range(len(t_end))]
+    te = [t_end[j] for _ in range(len(t_now)) for j in range(len(t_end))]
+    return np.asarray(tn, dtype=np.float32), np.asarray(te, dtype=np.float32)
