@@ -376,6 +376,34 @@ def run_e2e(torch, blk, inp, w, ws, steps, warmup, device):
             "overlap": "uploads, compute and downloads on three streams, double-buffered"}
 
 
+def run_modulation(torch, j, hi, device, peaks, steps):
+    """The modulation-table producer at real dimensions with two-time
+    conditioning (4 timestep sets, 4 modality tags): device time per call and
+    achieved HBM bandwidth over the bytes it must stream (every weight once,
+    the table written once)."""
+    from dataclasses import replace
+    dims, md = replace(hi.REAL, n_t=4), hi.REAL_MOD
+    p = hi.make_modulation_params(dims, md, two_time=True)
+    t_now, t_end = hi.two_time_sets([0.83, 0.41], [0.55, 0.12])
+    blk = j.H3Block(dims)
+    w = j.ModulationWeights(p, device)
+    for _ in range(3):
+        j.modulation_table(blk, w, t_now, t_end, 0.35)
+    torch.cuda.synchronize(device)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        j.modulation_table(blk, w, t_now, t_end, 0.35)
+    t1.record()
+    torch.cuda.synchronize(device)
+    ms = t0.elapsed_time(t1) / steps
+    mlp = 4 * (md.time_hidden * md.freq_dim + md.time_hidden + md.time_dim * md.time_hidden + md.time_dim)
+    nbytes = 2 * mlp + dims.n_tags * 6 * dims.hidden * (2 * md.time_dim + 4) + 4 * dims.n_tags * 4 * 6 * dims.hidden
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"ms": ms, "bytes": nbytes, "gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"],
+            "config": "real dims, 4 tags x 4 two-time sets, freq 256 -> 5376 -> 2688 -> 6 x 5376"}
+
+
 # --------------------------------------------------------------------------- CPU oracle arm
 
 def cpu_oracle_sample(name="t2va_32k", kv_rows=1024, q_rows=8, seed=0):
@@ -463,6 +491,7 @@ def main():
     w8 = None
     if not args.no_w8a8:
         w8 = run_gpu_case(torch, j, hi, "w8a8_t2va_32k", args.steps, args.warmup, device, peaks, int8_peak)
+    modt = run_modulation(torch, j, hi, device, peaks, args.steps)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rps, secs, desc, threads = cpu_oracle_sample(args.workload)
@@ -484,6 +513,7 @@ def main():
             line["w8a8"] = {"workload": w8["workload"], "value": w8["value"], "unit": UNIT,
                             "ms_per_step": w8["ms_per_step"], "roofline": w8["roofline"], "kernels": w8["kernels"],
                             "gpu_launches": w8["gpu_launches"]}
+        line["modulation_table"] = modt
         print(json.dumps(line), flush=True)
     import torch.distributed as dist
     if dist.is_initialized():

@@ -217,6 +217,43 @@ H3BLK_API int h3blk_gemm_s8_s32(int64_t M, int N, int K, const int8_t* A, const 
  * (K a multiple of 64, N a multiple of 128). */
 H3BLK_API int h3blk_gemm_bf16(int64_t M, int N, int K, const void* A, const void* B, void* C, void* stream);
 
+/* ------------------------------------------------- modulation-table producer */
+/* The step before the block: turns the distinct timesteps of a forward into the
+ * AdaLN table h3blk_forward reads.
+ *   e_k   = [cos(t_k w_i), sin(t_k w_i)], w_i = 10000^(-i / (freq_dim / 2)),
+ *           timesteps unscaled in [0, 1]
+ *   E_k   = (1 - g) (W2 silu(W1 e(t_now_k) + b1) + b2)
+ *           + g (W2r silu(W1r e(t_end_k) + b1r) + b2r)          (two-time blend)
+ *   table[tag][k] = A_tag silu(E_k) + a_tag  -> fp32 [n_tags][n_t][6][hidden]
+ * Sources: "MiniMaxH3Transformer3DModel" (diffusers API page), constructor
+ * (freq_dim, time_embed_hidden_dim, time_embed_dim) and introduction (the
+ * modality tag selects the AdaLN parameters; the timestep MLP is fp32);
+ * HyperFlow model card, "How it works" (second time embedder for the step
+ * endpoint, fixed blend gate; conditioning rows keep r = t). The embedding's
+ * channel order, the SiLU placements and the blend formula are readings. */
+typedef struct {
+  int freq_dim;     /* multiple of 16, <= 1024 (256 for the model) */
+  int time_hidden;  /* multiple of 8 (5376) */
+  int time_dim;     /* multiple of 8 (2688) */
+  const float *w1, *b1;      /* fp32 [time_hidden, freq_dim], [time_hidden]  */
+  const float *w2, *b2;      /* fp32 [time_dim, time_hidden], [time_dim]     */
+  const float *w1_r, *b1_r;  /* second-time copies; may be NULL when gate == 0 */
+  const float *w2_r, *b2_r;
+  const void* adaln_w;       /* bf16 [n_tags][6 * hidden][time_dim] */
+  const float* adaln_b;      /* fp32 [n_tags][6 * hidden]           */
+} h3blk_mod_weights;
+
+/* Scratch bytes h3blk_modulation_table needs (n_t * (time_hidden + time_dim) floats). */
+H3BLK_API int h3blk_modulation_scratch_bytes(h3blk_handle h, const h3blk_mod_weights* w, size_t* bytes);
+
+/* Writes the handle's n_t x n_tags table. t_now and t_end are HOST arrays of
+ * n_t timesteps (t_end may be NULL when gate == 0); n_t <= 8. Device pointers
+ * for weights, table and scratch. UNSUPPORTED when the sizes break the limits
+ * above or the inputs of one product exceed 200 KB of shared memory. */
+H3BLK_API int h3blk_modulation_table(h3blk_handle h, const h3blk_mod_weights* w, const float* t_now,
+                                     const float* t_end, float gate, float* table, void* scratch,
+                                     size_t scratch_bytes, void* stream);
+
 /* Document-masked attention of the block (the same kernels as the attention
  * step of h3blk_forward) for callers that cannot allocate device memory at run
  * time, such as a plugin inside a host application whose memory pool owns the

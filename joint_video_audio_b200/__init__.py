@@ -8,4 +8,6 @@ from ._binding import (  # noqa: F401
     EXPORTS, H3BLK_OK, H3BlkError, LIB_PATH, STAGE, STAGES, h3blk_config, h3blk_weights,
 )
 from . import _binding as capi  # noqa: F401
-from .block import DeviceWeights, H3Block, gemm_bf16, gemm_s8_s32, make_config, rotate_quantize  # noqa: F401
+from .block import (  # noqa: F401
+    DeviceWeights, H3Block, ModulationWeights, gemm_bf16, gemm_s8_s32, make_config, modulation_table, rotate_quantize,
+)

@@ -27,7 +27,8 @@ STAGE = {name: i for i, name in enumerate(STAGES)}
 EXPORTS = ["h3blk_create", "h3blk_destroy", "h3blk_workspace_bytes", "h3blk_stage_view", "h3blk_forward",
            "h3blk_check", "h3blk_int8_weights_bytes", "h3blk_prepare_int8_weights", "h3blk_rotate_quantize",
            "h3blk_gemm_s8_s32", "h3blk_gemm_bf16", "h3blk_error_string", "h3blk_version",
-           "h3blk_set_kernel_events", "h3blk_attention_noalloc"]
+           "h3blk_set_kernel_events", "h3blk_attention_noalloc", "h3blk_modulation_scratch_bytes",
+           "h3blk_modulation_table"]
 
 H3BLK_TIMING_POINTS = 11
 TIMING_INTERVALS = ["prep", "norm1", "qkv_gemm", "attention", "quant_o", "out_proj_gemm", "norm2",
@@ -45,6 +46,13 @@ class h3blk_weights(C.Structure):
     _fields_ = [("wqkv", C.c_void_p), ("q_gain", C.c_void_p), ("k_gain", C.c_void_p), ("wo", C.c_void_p),
                 ("w13", C.c_void_p), ("w2", C.c_void_p), ("s_qkv", C.c_void_p), ("s_o", C.c_void_p),
                 ("s_13", C.c_void_p), ("s_2", C.c_void_p)]
+
+
+class h3blk_mod_weights(C.Structure):
+    _fields_ = [("freq_dim", C.c_int), ("time_hidden", C.c_int), ("time_dim", C.c_int),
+                ("w1", C.c_void_p), ("b1", C.c_void_p), ("w2", C.c_void_p), ("b2", C.c_void_p),
+                ("w1_r", C.c_void_p), ("b1_r", C.c_void_p), ("w2_r", C.c_void_p), ("b2_r", C.c_void_p),
+                ("adaln_w", C.c_void_p), ("adaln_b", C.c_void_p)]
 
 
 class H3BlkError(RuntimeError):
@@ -74,6 +82,9 @@ def _load():
         "h3blk_version": (i32, []),
         "h3blk_set_kernel_events": (i32, [vp, C.POINTER(vp), i32]),
         "h3blk_attention_noalloc": (i32, [i64, i32, i32, i32, i32, vp, vp, vp, vp, vp]),
+        "h3blk_modulation_scratch_bytes": (i32, [vp, C.POINTER(h3blk_mod_weights), C.POINTER(sz)]),
+        "h3blk_modulation_table": (i32, [vp, C.POINTER(h3blk_mod_weights), C.POINTER(C.c_float),
+                                          C.POINTER(C.c_float), C.c_float, vp, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -187,3 +198,18 @@ def h3blk_attention_noalloc(n_rows, heads, head_dim, n_tags, n_t, qkv, tag, tidx
     """Raw call (pointers are ints); returns the status code. Uses the
     library's fixed device scratch instead of a caller workspace."""
     return _lib.h3blk_attention_noalloc(n_rows, heads, head_dim, n_tags, n_t, qkv, tag, tidx, o, stream)
+
+
+def h3blk_modulation_scratch_bytes(handle, w: h3blk_mod_weights) -> int:
+    n = C.c_size_t()
+    _check("h3blk_modulation_scratch_bytes", _lib.h3blk_modulation_scratch_bytes(handle, C.byref(w), C.byref(n)))
+    return n.value
+
+
+def h3blk_modulation_table(handle, w: h3blk_mod_weights, t_now, t_end, gate, table, scratch, scratch_bytes,
+                           stream) -> int:
+    """t_now / t_end: host sequences of floats (t_end may be None). Returns the status code."""
+    tn = (C.c_float * len(t_now))(*[float(v) for v in t_now])
+    te = (C.c_float * len(t_end))(*[float(v) for v in t_end]) if t_end is not None else None
+    return _lib.h3blk_modulation_table(handle, C.byref(w), tn, te, C.c_float(gate), table, scratch, scratch_bytes,
+                                       stream)

@@ -150,3 +150,33 @@ def gemm_bf16(a: torch.Tensor, b: torch.Tensor) -> torch.Tensor:
     if st != B.H3BLK_OK:
         raise B.H3BlkError("h3blk_gemm_bf16", st)
     return c
+
+
+# ---------------------------------------------------------------- modulation-table producer
+
+class ModulationWeights:
+    """Producer weights resident on the GPU and the C struct pointing at them."""
+
+    def __init__(self, p, device="cuda"):
+        """p: object with md (freq_dim, time_hidden, time_dim), fp32 w1, b1, w2,
+        b2 (and optional *_r copies), bf16 adaln_w, fp32 adaln_b."""
+        f32 = lambda t: None if t is None else t.to(device=device, dtype=torch.float32).contiguous()  # noqa: E731
+        self.t = {k: f32(getattr(p, k)) for k in ("w1", "b1", "w2", "b2", "w1_r", "b1_r", "w2_r", "b2_r", "adaln_b")}
+        self.t["adaln_w"] = p.adaln_w.to(device=device, dtype=torch.bfloat16).contiguous()
+        self.c = B.h3blk_mod_weights(freq_dim=p.md.freq_dim, time_hidden=p.md.time_hidden, time_dim=p.md.time_dim,
+                                     **{k: _ptr(v) for k, v in self.t.items()})
+
+
+def modulation_table(block: H3Block, w: ModulationWeights, t_now, t_end=None, gate=0.0, scratch=None):
+    """fp32 table [n_tags, n_t, 6, hidden] for h3blk_forward."""
+    d = block.dims
+    dev = w.t["w1"].device
+    table = torch.empty(d.n_tags, d.n_t, 6, d.hidden, dtype=torch.float32, device=dev)
+    nb = B.h3blk_modulation_scratch_bytes(block.handle, w.c)
+    if scratch is None:
+        scratch = torch.empty(nb, dtype=torch.uint8, device=dev)
+    st = B.h3blk_modulation_table(block.handle, w.c, list(t_now), None if t_end is None else list(t_end), gate,
+                                  table.data_ptr(), scratch.data_ptr(), scratch.numel(), _stream())
+    if st != B.H3BLK_OK:
+        raise B.H3BlkError("h3blk_modulation_table", st)
+    return table

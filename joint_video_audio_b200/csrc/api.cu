@@ -493,6 +493,72 @@ int h3blk_prepare_int8_weights(h3blk_handle h, const h3blk_weights* in, void* bl
   return H3BLK_OK;
 }
 
+static int mod_check(const h3blk_ctx* h, const h3blk_mod_weights* w) {
+  if (!h || !w) return H3BLK_ERR_INVALID_ARG;
+  if (w->freq_dim <= 0 || w->freq_dim % 16 || w->freq_dim > 1024 || w->time_hidden <= 0 || w->time_hidden % 8 ||
+      w->time_dim <= 0 || w->time_dim % 8 || h->cfg.n_t > h3::kMaxModSets)
+    return H3BLK_ERR_UNSUPPORTED;
+  const size_t biggest = (size_t)h->cfg.n_t * (size_t)(w->time_hidden > w->time_dim ? w->time_hidden : w->time_dim);
+  if (biggest * sizeof(float) > 200 * 1024) return H3BLK_ERR_UNSUPPORTED;
+  return H3BLK_OK;
+}
+
+int h3blk_modulation_scratch_bytes(h3blk_handle h, const h3blk_mod_weights* w, size_t* bytes) {
+  const int st = mod_check(h, w);
+  if (st != H3BLK_OK) return st;
+  if (!bytes) return H3BLK_ERR_INVALID_ARG;
+  *bytes = (size_t)h->cfg.n_t * (size_t)(w->time_hidden + w->time_dim) * sizeof(float);
+  return H3BLK_OK;
+}
+
+int h3blk_modulation_table(h3blk_handle h, const h3blk_mod_weights* w, const float* t_now, const float* t_end,
+                           float gate, float* table, void* scratch, size_t scratch_bytes, void* stream) {
+  int st = mod_check(h, w);
+  if (st != H3BLK_OK) return st;
+  const int V = h->cfg.n_t;
+  if (!t_now || !table || !scratch || !w->w1 || !w->b1 || !w->w2 || !w->b2 || !w->adaln_w || !w->adaln_b)
+    return H3BLK_ERR_INVALID_ARG;
+  if (!(gate >= 0.f && gate <= 1.f)) return H3BLK_ERR_INVALID_ARG;
+  if (gate != 0.f && (!t_end || !w->w1_r || !w->b1_r || !w->w2_r || !w->b2_r)) return H3BLK_ERR_INVALID_ARG;
+  if (scratch_bytes < (size_t)V * (size_t)(w->time_hidden + w->time_dim) * sizeof(float)) return H3BLK_ERR_INVALID_ARG;
+  const void* ptrs[] = {w->w1, w->w2, w->adaln_w, table, scratch};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return H3BLK_ERR_INVALID_ARG;
+  if (gate != 0.f && (!aligned16(w->w1_r) || !aligned16(w->w2_r))) return H3BLK_ERR_INVALID_ARG;
+  int sms = 0;
+  PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+  st = device_info(&sms, &enc);
+  if (st != H3BLK_OK) return st;
+  h3::ModTableArgs m;
+  std::memset(&m, 0, sizeof(m));
+  m.n_sets = V;
+  m.n_tags = h->cfg.n_tags;
+  m.hidden = h->cfg.hidden;
+  m.freq_dim = w->freq_dim;
+  m.time_hidden = w->time_hidden;
+  m.time_dim = w->time_dim;
+  m.t_now.count = V;
+  m.t_end.count = V;
+  for (int k = 0; k < V; ++k) {
+    m.t_now.t[k] = t_now[k];
+    m.t_end.t[k] = t_end ? t_end[k] : t_now[k];
+  }
+  m.gate = gate;
+  m.w1 = w->w1;
+  m.b1 = w->b1;
+  m.w2 = w->w2;
+  m.b2 = w->b2;
+  m.w1_r = w->w1_r;
+  m.b1_r = w->b1_r;
+  m.w2_r = w->w2_r;
+  m.b2_r = w->b2_r;
+  m.adaln_w = static_cast<const __nv_bfloat16*>(w->adaln_w);
+  m.adaln_b = w->adaln_b;
+  m.table = table;
+  m.scratch = static_cast<float*>(scratch);
+  return cuda_status(h3::launch_modulation_table(m, sms, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int h3blk_rotate_quantize(int64_t rows, int K, const void* in_bf16, int8_t* out_q, float* out_scale, void* stream) {
   if (rows < 0 || K <= 0 || K % 128 || K > 16384 || !in_bf16 || !out_q || !out_scale) return H3BLK_ERR_INVALID_ARG;
   if (!aligned16(in_bf16) || !aligned16(out_q) || !aligned16(out_scale)) return H3BLK_ERR_INVALID_ARG;

@@ -109,4 +109,25 @@ struct AttnArgs {
 };
 cudaError_t launch_attention(const AttnArgs& a, PFN_cuTensorMapEncodeTiled_v12000 encode, cudaStream_t s);
 
+// ---------------------------------------------------------------- modulation table
+constexpr int kMaxModSets = 8;  // timestep sets (the table's n_t) per call
+
+struct ModTimes {
+  int count;                 // 0: no embedding (the input comes from memory)
+  float t[kMaxModSets];
+};
+
+struct ModTableArgs {
+  int n_sets, n_tags, hidden, freq_dim, time_hidden, time_dim;
+  ModTimes t_now, t_end;     // per set
+  float gate;                // two-time blend weight of the t_end embedding
+  const float *w1, *b1, *w2, *b2;
+  const float *w1_r, *b1_r, *w2_r, *b2_r;
+  const __nv_bfloat16* adaln_w;  // [n_tags][6 * hidden][time_dim]
+  const float* adaln_b;          // [n_tags][6 * hidden]
+  float* table;              // [n_tags][n_sets][6 * hidden]
+  float* scratch;            // n_sets * (time_hidden + time_dim) floats
+};
+cudaError_t launch_modulation_table(const ModTableArgs& a, int num_sms, cudaStream_t s);
+
 }  // namespace h3

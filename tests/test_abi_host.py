@@ -149,3 +149,25 @@ def test_kernel_level_calls_reject_bad_sizes():
     assert B.h3blk_gemm_s8_s32(16, 128, 64, 1 << 40, 1 << 41, 1 << 42, None) == B.H3BLK_ERR_INVALID_ARG
     assert B.h3blk_gemm_bf16(16, 128, 32, 1 << 40, 1 << 41, 1 << 42, None) == B.H3BLK_ERR_INVALID_ARG
     assert B.h3blk_gemm_bf16(16, 128, 64, 0, 1 << 41, 1 << 42, None) == B.H3BLK_ERR_INVALID_ARG
+
+
+def test_modulation_producer_validation_before_gpu():
+    blk = j.H3Block(hi.TINY)
+    base = 1 << 40
+    w = B.h3blk_mod_weights(freq_dim=64, time_hidden=128, time_dim=64, w1=base, b1=base, w2=base, b2=base,
+                            adaln_w=base, adaln_b=base)
+    assert B.h3blk_modulation_scratch_bytes(blk.handle, w) == hi.TINY.n_t * (128 + 64) * 4
+    # bad sizes
+    w_bad = B.h3blk_mod_weights(freq_dim=60, time_hidden=128, time_dim=64)
+    assert B.h3blk_modulation_table(blk.handle, w_bad, [0.1, 0.2], None, 0.0, base, base, 1 << 20,
+                                    None) == B.H3BLK_ERR_UNSUPPORTED
+    # missing second-time weights with a non-zero gate
+    assert B.h3blk_modulation_table(blk.handle, w, [0.1, 0.2], [0.0, 0.0], 0.5, base, base, 1 << 20,
+                                    None) == B.H3BLK_ERR_INVALID_ARG
+    # gate outside [0, 1], scratch too small, null table
+    assert B.h3blk_modulation_table(blk.handle, w, [0.1, 0.2], None, 1.5, base, base, 1 << 20, None) == \
+        B.H3BLK_ERR_INVALID_ARG
+    assert B.h3blk_modulation_table(blk.handle, w, [0.1, 0.2], None, 0.0, base, base, 16, None) == \
+        B.H3BLK_ERR_INVALID_ARG
+    assert B.h3blk_modulation_table(blk.handle, w, [0.1, 0.2], None, 0.0, 0, base, 1 << 20, None) == \
+        B.H3BLK_ERR_INVALID_ARG
