@@ -386,3 +386,134 @@ def two_time_sets(t_now, t_end):
     tn = [t_now[i] for i in range(len(t_now)) for _ in range(len(t_end))]
     te = [t_end[j] for _ in range(len(t_now)) for j in range(len(t_end))]
     return np.asarray(tn, dtype=np.float32), np.asarray(te, dtype=np.float32)
+
+
+# --------------------------------------------------------------------------
+# Model shell around the block stack
+# ("MiniMaxH3Transformer3DModel", constructor: num_layers, num_refiner_layers,
+# in_channels x patch_size, audio_in_channels, text_dim, final_norm_eps;
+# forward: video_indices, audio_indices, text_indices)
+# --------------------------------------------------------------------------
+
+@dataclass(frozen=True)
+class ShellDims:
+    video_in: int = 96       # in_channels 24 x patch (1, 2, 2)
+    audio_in: int = 32
+    text_dim: int = 5120
+    n_layers: int = 50
+    n_refiner: int = 2
+    final_norm_eps: float = 1e-5
+
+
+REAL_SHELL = ShellDims()
+TINY_SHELL = ShellDims(video_in=16, audio_in=8, text_dim=128, n_layers=2, n_refiner=1)
+
+
+@dataclass
+class Layer:
+    """One block of the stack with its AdaLN projection."""
+    w: Weights
+    adaln_w: torch.Tensor   # bf16 [n_tags, 6C, time_dim]
+    adaln_b: torch.Tensor   # fp32 [n_tags, 6C]
+
+
+@dataclass
+class ModelParams:
+    sd: ShellDims
+    time: ModParams             # time MLP; its adaln_w / adaln_b are not used by the model
+    layers: list                # [Layer] * n_layers
+    refiner: list               # [Layer] * n_refiner
+    refiner_gain: torch.Tensor  # bf16 [C]
+    out_adaln_w: torch.Tensor   # bf16 [n_tags, 2C, time_dim]
+    out_adaln_b: torch.Tensor   # fp32 [n_tags, 2C]
+    proj_in_w: torch.Tensor     # fp32 [C, video_in]
+    proj_in_b: torch.Tensor     # fp32 [C]
+    audio_in_w: torch.Tensor    # fp32 [C, audio_in]
+    audio_in_b: torch.Tensor    # fp32 [C]
+    ctx_w: torch.Tensor         # bf16 [C, text_dim]
+    ctx_b: torch.Tensor         # fp32 [C]
+    proj_out_w: torch.Tensor    # fp32 [video_in, C]
+    proj_out_b: torch.Tensor    # fp32 [video_in]
+    audio_out_w: torch.Tensor   # fp32 [audio_in, C]
+    audio_out_b: torch.Tensor   # fp32 [audio_in]
+
+
+def _adaln(rng, dims: Dims, md: ModDims, n_vec: int):
+    aw = to_bf16(_normal(rng, (dims.n_tags, n_vec * dims.hidden, md.time_dim), 0.1 / np.sqrt(md.time_dim)))
+    ab = torch.from_numpy(_normal(rng, (dims.n_tags, n_vec * dims.hidden), 0.02))
+    return aw, ab
+
+
+def make_model_params(dims: Dims, md: ModDims, sd: ShellDims, seed=0, two_time=False) -> ModelParams:
+    """Every weight ~ N(0, 1/fan_in) (AdaLN projections 0.1/sqrt(fan_in)),
+    biases N(0, 0.02^2), the refiner's output-norm gain 1 + N(0, 0.1^2)."""
+    time = make_modulation_params(dims, md, seed, two_time)
+    rng = np.random.default_rng(seed + 60)
+    C = dims.hidden
+    f = lambda a: torch.from_numpy(a)  # noqa: E731
+
+    def layer(k):
+        aw, ab = _adaln(rng, dims, md, 6)
+        return Layer(make_weights(dims, seed + 1000 * (k + 1)), aw, ab)
+    layers = [layer(k) for k in range(sd.n_layers)]
+    refiner = [layer(100 + k) for k in range(sd.n_refiner)]
+    oaw, oab = _adaln(rng, dims, md, 2)
+    return ModelParams(
+        sd, time, layers, refiner,
+        refiner_gain=to_bf16(1.0 + _normal(rng, (C,), 0.1)),
+        out_adaln_w=oaw, out_adaln_b=oab,
+        proj_in_w=f(_normal(rng, (C, sd.video_in), 1.0 / np.sqrt(sd.video_in))),
+        proj_in_b=f(_normal(rng, (C,), 0.02)),
+        audio_in_w=f(_normal(rng, (C, sd.audio_in), 1.0 / np.sqrt(sd.audio_in))),
+        audio_in_b=f(_normal(rng, (C,), 0.02)),
+        ctx_w=to_bf16(_normal(rng, (C, sd.text_dim), 1.0 / np.sqrt(sd.text_dim))),
+        ctx_b=f(_normal(rng, (C,), 0.02)),
+        proj_out_w=f(_normal(rng, (sd.video_in, C), 1.0 / np.sqrt(C))),
+        proj_out_b=f(_normal(rng, (sd.video_in,), 0.02)),
+        audio_out_w=f(_normal(rng, (sd.audio_in, C), 1.0 / np.sqrt(C))),
+        audio_out_b=f(_normal(rng, (sd.audio_in,), 0.02)))
+
+
+def model_indices(layout: Layout):
+    """(video, audio, text) row indices of a packed layout: video rows are the
+    target-video and conditioning (image / video reference) rows, audio rows
+    every audio-tagged row, text rows the text-tagged ones; padding rows are in
+    none of them. Each list is in sequence order."""
+    t = layout.tag
+    video = np.nonzero((t == TAG_VIDEO) | (t == TAG_COND))[0].astype(np.int32)
+    audio = np.nonzero(t == TAG_AUDIO)[0].astype(np.int32)
+    text = np.nonzero(t == TAG_TEXT)[0].astype(np.int32)
+    return video, audio, text
+
+
+@dataclass
+class ModelInputs:
+    layout: Layout
+    video_idx: np.ndarray   # int32 [Nv]
+    audio_idx: np.ndarray   # int32 [Na]
+    text_idx: np.ndarray    # int32 [Nt]
+    video: torch.Tensor     # fp32 [Nv, video_in], patchified latent rows
+    audio: torch.Tensor     # fp32 [Na, audio_in]
+    text: torch.Tensor      # bf16 [Nt, text_dim], text-encoder states
+    t_now: np.ndarray       # fp32 [n_t], per modulation set
+    t_end: np.ndarray       # fp32 [n_t]
+    gate: float
+
+
+def make_model_inputs(dims: Dims, sd: ShellDims, layout: Layout, seed=0, two_time=False,
+                      gate=0.35) -> ModelInputs:
+    """Latent rows ~ N(0, 1), text states ~ N(0, 1) in bf16; timesteps drawn
+    uniformly in [0, 1] per set (two-time: t_now pairs, t_end pairs, expanded
+    to the 2 i + j sets)."""
+    rng = np.random.default_rng(seed + 70)
+    v, a, t = model_indices(layout)
+    video = torch.from_numpy(_normal(rng, (v.size, sd.video_in), 1.0))
+    audio = torch.from_numpy(_normal(rng, (a.size, sd.audio_in), 1.0))
+    text = to_bf16(_normal(rng, (t.size, sd.text_dim), 1.0))
+    if two_time:
+        assert dims.n_t == 4
+        tn, te = two_time_sets(rng.uniform(0, 1, 2).astype(np.float32), rng.uniform(0, 1, 2).astype(np.float32))
+    else:
+        tn = rng.uniform(0, 1, dims.n_t).astype(np.float32)
+        te, gate = tn.copy(), 0.0
+    return ModelInputs(layout, v, a, t, video, audio, text, tn, te, float(gate))

@@ -9,3 +9,7 @@ from .h3_block import (  # noqa: F401
     rope_angles, rope_frequencies, rotate_blocks, silu, softmax, swiglu,
     sylvester_hadamard, w8a8_linear,
 )
+from .h3_modulation import (  # noqa: F401
+    modulation_table, produce, sinusoidal_embedding, time_mlp, timestep_frequencies, two_time_embedding,
+)
+from .h3_model import ModelOracle, affine, norm_out, refine_text, scatter_rows  # noqa: F401

@@ -65,14 +65,15 @@ def f64(t):
 # --------------------------------------------------------------------------
 
 def modulation(table, tag, tidx):
-    """Per-row modulation vectors m[r] = table[tag[r]][tidx[r]] ([R, 6, C]);
+    """Per-row modulation vectors m[r] = table[tag[r]][tidx[r]] ([R, 6, C] for
+    a block's table, [R, 2, C] for norm_out's);
     zero for padding rows, which have no table row.
     ("MiniMaxH3Transformer3DModel", introduction: the per-row modality tag
     selects the AdaLN modulation parameters; forward: timestep_indices.)"""
     table = f64(table)
     tag = np.asarray(tag)
     tidx = np.asarray(tidx)
-    m = np.zeros((tag.shape[0], 6, table.shape[-1]), dtype=np.float64)
+    m = np.zeros((tag.shape[0],) + table.shape[2:], dtype=np.float64)
     valid = tag != TAG_PAD
     m[valid] = table[tag[valid], tidx[valid]]
     return m
