@@ -254,6 +254,102 @@ H3BLK_API int h3blk_modulation_table(h3blk_handle h, const h3blk_mod_weights* w,
                                      const float* t_end, float gate, float* table, void* scratch,
                                      size_t scratch_bytes, void* stream);
 
+/* ------------------------------------------------------------ model shell */
+/* The whole transformer forward around the block ("MiniMaxH3Transformer3DModel",
+ * diffusers API page: introduction, constructor and forward parameters):
+ *
+ *   x[video_idx] = proj_in(video)            fp32 W [hidden, video_in] + b
+ *   x[audio_idx] = audio_proj_in(audio)      fp32 W [hidden, audio_in] + b
+ *   r = context_embedder(text)               bf16 W [hidden, text_dim] + fp32 b
+ *   r = refiner layers over the text rows alone (the same block, each row with
+ *       its packed tag / tidx / position), then rmsnorm(r, final_eps) * gain
+ *   x[text_idx] = r; every other row (padding) = 0
+ *   x = layer_{L-1}( ... layer_0(x))         h3blk_forward per layer
+ *   h = rmsnorm(x, final_eps) (1 + scale_o) + shift_o     (norm_out)
+ *   video_out = proj_out(h[video_idx]);  audio_out = audio_proj_out(h[audio_idx])
+ *
+ * Every layer (stack and refiner) owns its AdaLN projection; all of them and
+ * norm_out's read the one time embedding of the forward's timestep sets
+ * (h3blk_modulation_table's first half). The refiner always runs the bf16
+ * block; the stack runs the handle's mode (bf16 or W8A8). The affine form of
+ * the projections, the refiner's block structure and output norm, and the
+ * AdaLN form of norm_out are readings: the pages name the modules only. */
+typedef struct {
+  int n_layers;        /* blocks of the stack (50; 47 in the pruned variant) */
+  int n_refiner;       /* token-refiner blocks (2) */
+  int video_in;        /* in_channels * prod(patch_size) (96); multiple of 4, <= 128 */
+  int audio_in;        /* audio_in_channels (32); multiple of 4, <= 128 */
+  int text_dim;        /* text_dim (5120); multiple of 64 */
+  float final_norm_eps;
+} h3blk_model_config;
+
+typedef struct {
+  h3blk_weights w;     /* the block's linears (bf16, or the int8 blob's pointers for the W8A8 stack) */
+  const void* adaln_w; /* bf16 [n_tags][6 * hidden][time_dim] */
+  const float* adaln_b; /* fp32 [n_tags][6 * hidden] */
+} h3blk_layer_weights;
+
+typedef struct {
+  h3blk_mod_weights time;            /* time MLP (+ r copy); its adaln_w / adaln_b are not read */
+  const h3blk_layer_weights* layers;  /* HOST array of n_layers entries */
+  const h3blk_layer_weights* refiner; /* HOST array of n_refiner entries (bf16 weights) */
+  const void* refiner_gain;          /* bf16 [hidden] */
+  const void* out_adaln_w;           /* bf16 [n_tags][2 * hidden][time_dim]: shift, scale */
+  const float* out_adaln_b;          /* fp32 [n_tags][2 * hidden] */
+  const float *proj_in_w, *proj_in_b;     /* fp32 [hidden][video_in], [hidden] */
+  const float *audio_in_w, *audio_in_b;   /* fp32 [hidden][audio_in], [hidden] */
+  const void* ctx_w;                      /* bf16 [hidden][text_dim] */
+  const float* ctx_b;                     /* fp32 [hidden] */
+  const float *proj_out_w, *proj_out_b;   /* fp32 [video_in][hidden], [video_in] */
+  const float *audio_out_w, *audio_out_b; /* fp32 [audio_in][hidden], [audio_in] */
+} h3blk_model_weights;
+
+/* One packed sequence. Every pointer is device memory. The three index
+ * tensors address distinct rows of [0, n_rows); rows none of them addresses
+ * must carry tag -1 (padding). An index outside [0, n_rows) is skipped and
+ * reported by h3blk_model_check as H3BLK_ERR_BAD_INDEX; rows addressed twice
+ * get one of the writers (unspecified which). Counts may be 0. */
+typedef struct {
+  int64_t n_rows, n_video, n_audio, n_text;
+  const int32_t *tag, *tidx, *pos;          /* [n_rows], [n_rows], [n_rows][3] */
+  const int32_t *video_idx, *audio_idx, *text_idx;
+  const float* video;   /* fp32 [n_video][video_in] patchified latent rows */
+  const float* audio;   /* fp32 [n_audio][audio_in] */
+  const void* text;     /* bf16 [n_text][text_dim] text-encoder states */
+  const float* t_now;   /* fp32 [n_t] per modulation set, in [0, 1] */
+  const float* t_end;   /* fp32 [n_t]; may be NULL when gate == 0 */
+  float gate;           /* two-time blend weight, in [0, 1] */
+} h3blk_model_inputs;
+
+/* Workspace bytes of a model forward over n_rows packed rows of which n_text
+ * are text rows. */
+H3BLK_API int h3blk_model_workspace_bytes(h3blk_handle h, const h3blk_model_config* mc, const h3blk_mod_weights* time,
+                                          int64_t n_rows, int64_t n_text, size_t* bytes);
+
+/* The forward, asynchronous on `stream`: video_out fp32 [n_video][video_in],
+ * audio_out fp32 [n_audio][audio_in]. Host-side checks only; device-side
+ * errors (bad indices, timeouts) are read by h3blk_model_check. */
+H3BLK_API int h3blk_model_forward(h3blk_handle h, const h3blk_model_config* mc, const h3blk_model_weights* w,
+                                  const h3blk_model_inputs* in, float* video_out, float* audio_out, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, then reads the error word a model forward left in
+ * `workspace` (sticky over all its layers). */
+H3BLK_API int h3blk_model_check(const void* workspace, void* stream, int* status);
+
+/* CUDA graph of one model forward: the same launches as h3blk_model_forward,
+ * captured once on a private stream (no work runs during capture) and
+ * instantiated. Every pointer of `w`, `in` and the outputs is baked into the
+ * graph: to run another step, write the new latents, text states and
+ * timesteps into the same device buffers and launch the graph again. The
+ * caller keeps all of those buffers alive until h3blk_graph_destroy. */
+typedef struct h3blk_graph_s* h3blk_graph;
+H3BLK_API int h3blk_model_graph_create(h3blk_handle h, const h3blk_model_config* mc, const h3blk_model_weights* w,
+                                       const h3blk_model_inputs* in, float* video_out, float* audio_out,
+                                       void* workspace, size_t workspace_bytes, h3blk_graph* out);
+H3BLK_API int h3blk_graph_launch(h3blk_graph g, void* stream);
+H3BLK_API void h3blk_graph_destroy(h3blk_graph g);
+
 /* Document-masked attention of the block (the same kernels as the attention
  * step of h3blk_forward) for callers that cannot allocate device memory at run
  * time, such as a plugin inside a host application whose memory pool owns the

@@ -28,7 +28,8 @@ EXPORTS = ["h3blk_create", "h3blk_destroy", "h3blk_workspace_bytes", "h3blk_stag
            "h3blk_check", "h3blk_int8_weights_bytes", "h3blk_prepare_int8_weights", "h3blk_rotate_quantize",
            "h3blk_gemm_s8_s32", "h3blk_gemm_bf16", "h3blk_error_string", "h3blk_version",
            "h3blk_set_kernel_events", "h3blk_attention_noalloc", "h3blk_modulation_scratch_bytes",
-           "h3blk_modulation_table"]
+           "h3blk_modulation_table", "h3blk_model_workspace_bytes", "h3blk_model_forward", "h3blk_model_check",
+           "h3blk_model_graph_create", "h3blk_graph_launch", "h3blk_graph_destroy"]
 
 H3BLK_TIMING_POINTS = 11
 TIMING_INTERVALS = ["prep", "norm1", "qkv_gemm", "attention", "quant_o", "out_proj_gemm", "norm2",
@@ -53,6 +54,34 @@ class h3blk_mod_weights(C.Structure):
                 ("w1", C.c_void_p), ("b1", C.c_void_p), ("w2", C.c_void_p), ("b2", C.c_void_p),
                 ("w1_r", C.c_void_p), ("b1_r", C.c_void_p), ("w2_r", C.c_void_p), ("b2_r", C.c_void_p),
                 ("adaln_w", C.c_void_p), ("adaln_b", C.c_void_p)]
+
+
+class h3blk_model_config(C.Structure):
+    _fields_ = [("n_layers", C.c_int), ("n_refiner", C.c_int), ("video_in", C.c_int), ("audio_in", C.c_int),
+                ("text_dim", C.c_int), ("final_norm_eps", C.c_float)]
+
+
+class h3blk_layer_weights(C.Structure):
+    _fields_ = [("w", h3blk_weights), ("adaln_w", C.c_void_p), ("adaln_b", C.c_void_p)]
+
+
+class h3blk_model_weights(C.Structure):
+    _fields_ = [("time", h3blk_mod_weights), ("layers", C.POINTER(h3blk_layer_weights)),
+                ("refiner", C.POINTER(h3blk_layer_weights)), ("refiner_gain", C.c_void_p),
+                ("out_adaln_w", C.c_void_p), ("out_adaln_b", C.c_void_p),
+                ("proj_in_w", C.c_void_p), ("proj_in_b", C.c_void_p),
+                ("audio_in_w", C.c_void_p), ("audio_in_b", C.c_void_p),
+                ("ctx_w", C.c_void_p), ("ctx_b", C.c_void_p),
+                ("proj_out_w", C.c_void_p), ("proj_out_b", C.c_void_p),
+                ("audio_out_w", C.c_void_p), ("audio_out_b", C.c_void_p)]
+
+
+class h3blk_model_inputs(C.Structure):
+    _fields_ = [("n_rows", C.c_int64), ("n_video", C.c_int64), ("n_audio", C.c_int64), ("n_text", C.c_int64),
+                ("tag", C.c_void_p), ("tidx", C.c_void_p), ("pos", C.c_void_p),
+                ("video_idx", C.c_void_p), ("audio_idx", C.c_void_p), ("text_idx", C.c_void_p),
+                ("video", C.c_void_p), ("audio", C.c_void_p), ("text", C.c_void_p),
+                ("t_now", C.c_void_p), ("t_end", C.c_void_p), ("gate", C.c_float)]
 
 
 class H3BlkError(RuntimeError):
@@ -85,6 +114,15 @@ def _load():
         "h3blk_modulation_scratch_bytes": (i32, [vp, C.POINTER(h3blk_mod_weights), C.POINTER(sz)]),
         "h3blk_modulation_table": (i32, [vp, C.POINTER(h3blk_mod_weights), C.POINTER(C.c_float),
                                           C.POINTER(C.c_float), C.c_float, vp, vp, sz, vp]),
+        "h3blk_model_workspace_bytes": (i32, [vp, C.POINTER(h3blk_model_config), C.POINTER(h3blk_mod_weights),
+                                               i64, i64, C.POINTER(sz)]),
+        "h3blk_model_forward": (i32, [vp, C.POINTER(h3blk_model_config), C.POINTER(h3blk_model_weights),
+                                       C.POINTER(h3blk_model_inputs), vp, vp, vp, sz, vp]),
+        "h3blk_model_check": (i32, [vp, vp, C.POINTER(i32)]),
+        "h3blk_model_graph_create": (i32, [vp, C.POINTER(h3blk_model_config), C.POINTER(h3blk_model_weights),
+                                            C.POINTER(h3blk_model_inputs), vp, vp, vp, sz, C.POINTER(vp)]),
+        "h3blk_graph_launch": (i32, [vp, vp]),
+        "h3blk_graph_destroy": (None, [vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -213,3 +251,38 @@ def h3blk_modulation_table(handle, w: h3blk_mod_weights, t_now, t_end, gate, tab
     te = (C.c_float * len(t_end))(*[float(v) for v in t_end]) if t_end is not None else None
     return _lib.h3blk_modulation_table(handle, C.byref(w), tn, te, C.c_float(gate), table, scratch, scratch_bytes,
                                        stream)
+
+
+def h3blk_model_workspace_bytes(handle, mc: h3blk_model_config, time: h3blk_mod_weights, n_rows, n_text) -> int:
+    n = C.c_size_t()
+    _check("h3blk_model_workspace_bytes",
+           _lib.h3blk_model_workspace_bytes(handle, C.byref(mc), C.byref(time), n_rows, n_text, C.byref(n)))
+    return n.value
+
+
+def h3blk_model_forward(handle, mc, w, inp, video_out, audio_out, workspace, workspace_bytes, stream) -> int:
+    """Raw call (pointers are ints); returns the status code."""
+    return _lib.h3blk_model_forward(handle, C.byref(mc), C.byref(w), C.byref(inp), video_out, audio_out, workspace,
+                                    workspace_bytes, stream)
+
+
+def h3blk_model_check(workspace, stream) -> int:
+    st = C.c_int()
+    _check("h3blk_model_check", _lib.h3blk_model_check(workspace, stream, C.byref(st)))
+    return st.value
+
+
+def h3blk_model_graph_create(handle, mc, w, inp, video_out, audio_out, workspace, workspace_bytes) -> int:
+    g = C.c_void_p()
+    _check("h3blk_model_graph_create",
+           _lib.h3blk_model_graph_create(handle, C.byref(mc), C.byref(w), C.byref(inp), video_out, audio_out,
+                                         workspace, workspace_bytes, C.byref(g)))
+    return g.value
+
+
+def h3blk_graph_launch(graph, stream) -> int:
+    return _lib.h3blk_graph_launch(graph, stream)
+
+
+def h3blk_graph_destroy(graph) -> None:
+    _lib.h3blk_graph_destroy(graph)

@@ -9,14 +9,12 @@
 #include <mutex>
 #include <new>
 
-#include "../../include/h3blk.h"
-#include "kernels.cuh"
+#include "api_internal.h"
 #include "ptx.cuh"
 
 using h3::GemmArgs;
 
 namespace {
-
 constexpr int kVersion = 100;  // 0.1.0
 
 // ------------------------------------------------------------------ device info
@@ -28,8 +26,10 @@ constexpr int kMaxDevices = 64;
 DeviceInfo g_dev[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::mutex g_mu;
+}  // namespace
 
-// Current device's SM count and the driver's tensor-map encoder.
+namespace h3api {
+
 int device_info(int* num_sms, PFN_cuTensorMapEncodeTiled_v12000* encode) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return H3BLK_ERR_CUDA;
@@ -62,23 +62,20 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? H3BLK_OK : H3BLK_ERR_
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+}  // namespace h3api
+
+namespace {
+using h3api::aligned16;
+using h3api::align256;
+using h3api::cuda_status;
+using h3api::device_info;
+
 bool overlap(const void* a, size_t na, const void* b, size_t nb) {
   const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
   return x < y + nb && y < x + na;
 }
-
-size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
-
-}  // namespace
-
-struct h3blk_ctx {
-  h3blk_config cfg;
-  h3::RopeTable rope;
-  cudaEvent_t events[H3BLK_TIMING_POINTS];
-  bool timing;
-};
-
-namespace {
 
 // Workspace layout: every stage buffer at a 256-byte aligned offset.
 struct Layout {
@@ -166,110 +163,26 @@ GemmArgs base_gemm(const h3blk_ctx* h, int* err) {
 
 }  // namespace
 
-extern "C" {
+namespace h3api {
 
-const char* h3blk_error_string(int status) {
-  switch (status) {
-    case H3BLK_OK: return "ok";
-    case H3BLK_ERR_INVALID_ARG: return "invalid argument (null or misaligned pointer, bad size, or aliasing)";
-    case H3BLK_ERR_UNSUPPORTED: return "unsupported dimension or device";
-    case H3BLK_ERR_CUDA: return "CUDA runtime or driver error";
-    case H3BLK_ERR_TIMEOUT: return "a kernel pipeline wait timed out";
-    case H3BLK_ERR_BAD_INDEX: return "a modality tag or timestep index lies outside the modulation table";
-    default: return "unknown status";
-  }
-}
-
-int h3blk_version(void) { return kVersion; }
-
-int h3blk_create(const h3blk_config* cfg, h3blk_handle* out) {
-  if (!cfg || !out) return H3BLK_ERR_INVALID_ARG;
-  *out = nullptr;
-  const h3blk_config& c = *cfg;
-  if (c.hidden <= 0 || c.heads <= 0 || c.head_dim <= 0 || c.ffn <= 0 || c.n_tags <= 0 || c.n_t <= 0 ||
-      c.rope_pairs_t < 0 || c.rope_pairs_h < 0 || c.rope_pairs_w < 0 || !(c.rope_theta > 0.f) ||
-      !(c.norm_eps >= 0.f) || !(c.qk_norm_eps >= 0.f) || (c.quant != 0 && c.quant != 1))
-    return H3BLK_ERR_INVALID_ARG;
-  if (c.hidden % 128 || c.ffn % 128 || (c.head_dim != 64 && c.head_dim != 128) || (c.heads * c.head_dim) % 128 ||
-      c.rope_pairs_t + c.rope_pairs_h + c.rope_pairs_w > c.head_dim / 2 || c.hidden > 6144 || c.ffn > 16384 ||
-      c.heads * c.head_dim > 16384)
-    return H3BLK_ERR_UNSUPPORTED;
-  h3blk_ctx* h = new (std::nothrow) h3blk_ctx;
-  if (!h) return H3BLK_ERR_INVALID_ARG;
-  h->cfg = c;
-  h->timing = false;
-  for (auto& e : h->events) e = nullptr;
-  const int pairs[3] = {c.rope_pairs_t, c.rope_pairs_h, c.rope_pairs_w};
-  int j = 0;
-  for (int axis = 0; axis < 3; ++axis)
-    for (int i = 0; i < pairs[axis]; ++i, ++j) {
-      h->rope.axis[j] = (int8_t)axis;
-      h->rope.freq[j] = (float)std::pow((double)c.rope_theta, -(double)i / (double)pairs[axis]);
-    }
-  for (; j < h3::kMaxRopePairs; ++j) {
-    h->rope.axis[j] = 3;
-    h->rope.freq[j] = 0.f;
-  }
-  *out = h;
-  return H3BLK_OK;
-}
-
-void h3blk_destroy(h3blk_handle h) { delete h; }
-
-int h3blk_set_kernel_events(h3blk_handle h, void* const* events, int n_events) {
-  if (!h) return H3BLK_ERR_INVALID_ARG;
-  if (n_events == 0 || !events) {
-    h->timing = false;
-    return H3BLK_OK;
-  }
-  if (n_events != H3BLK_TIMING_POINTS) return H3BLK_ERR_INVALID_ARG;
-  for (int i = 0; i < n_events; ++i) {
-    if (!events[i]) return H3BLK_ERR_INVALID_ARG;
-    h->events[i] = reinterpret_cast<cudaEvent_t>(events[i]);
-  }
-  h->timing = true;
-  return H3BLK_OK;
-}
-
-int h3blk_workspace_bytes(h3blk_handle h, int64_t n_rows, size_t* bytes) {
-  if (!h || !bytes || n_rows < 1) return H3BLK_ERR_INVALID_ARG;
-  *bytes = make_layout(h->cfg, n_rows).total;
-  return H3BLK_OK;
-}
-
-int h3blk_stage_view(h3blk_handle h, int64_t n_rows, int stage, size_t* offset, size_t* bytes) {
-  if (!h || !offset || !bytes || n_rows < 1 || stage < 0 || stage >= H3BLK_STAGE_COUNT) return H3BLK_ERR_INVALID_ARG;
-  const Layout L = make_layout(h->cfg, n_rows);
-  if (L.len[stage] == 0) return H3BLK_ERR_UNSUPPORTED;  // stage not produced in this mode
-  *offset = L.off[stage];
-  *bytes = L.len[stage];
-  return H3BLK_OK;
-}
-
-int h3blk_forward(h3blk_handle h, int64_t n_rows, const void* x, const int32_t* tag, const int32_t* tidx,
-                  const int32_t* pos, const float* mod_table, const h3blk_weights* w, void* out, void* workspace,
-                  size_t workspace_bytes, void* stream) {
-  if (!h || !w || n_rows < 1 || !x || !tag || !tidx || !pos || !mod_table || !out || !workspace)
-    return H3BLK_ERR_INVALID_ARG;
-  const h3blk_config& c = h->cfg;
-  const bool q = c.quant != 0;
-  if (!w->wqkv || !w->q_gain || !w->k_gain || !w->wo || !w->w13 || !w->w2) return H3BLK_ERR_INVALID_ARG;
-  if (q && (!w->s_qkv || !w->s_o || !w->s_13 || !w->s_2)) return H3BLK_ERR_INVALID_ARG;
-  const void* ptrs[] = {x, tag, tidx, pos, mod_table, out, workspace, w->wqkv, w->wo, w->w13, w->w2};
+int check_block_weights(const h3blk_config& c, const h3blk_weights* w) {
+  if (!w || !w->wqkv || !w->q_gain || !w->k_gain || !w->wo || !w->w13 || !w->w2) return H3BLK_ERR_INVALID_ARG;
+  if (c.quant != 0 && (!w->s_qkv || !w->s_o || !w->s_13 || !w->s_2)) return H3BLK_ERR_INVALID_ARG;
+  const void* ptrs[] = {w->wqkv, w->wo, w->w13, w->w2};
   for (const void* p : ptrs)
     if (!aligned16(p)) return H3BLK_ERR_INVALID_ARG;
-  const Layout L = make_layout(c, n_rows);
-  if (workspace_bytes < L.total) return H3BLK_ERR_INVALID_ARG;
-  const size_t N = (size_t)n_rows, C = c.hidden, HD = (size_t)c.heads * c.head_dim, F = c.ffn;
-  if (overlap(out, N * C * 2, x, N * C * 2) || overlap(out, N * C * 2, workspace, L.total) ||
-      overlap(x, N * C * 2, workspace, L.total))
-    return H3BLK_ERR_INVALID_ARG;
-  int sms = 0;
-  PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
-  int st = device_info(&sms, &enc);
-  if (st != H3BLK_OK) return st;
+  return H3BLK_OK;
+}
 
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+size_t block_workspace_bytes(const h3blk_config& c, int64_t n) { return make_layout(c, n).total; }
+
+int block_forward(const h3blk_ctx* h, int64_t n_rows, const void* x, const int32_t* tag, const int32_t* tidx,
+                  const int32_t* pos, const float* mod_table, const h3blk_weights* w, void* out, void* workspace,
+                  int sms, PFN_cuTensorMapEncodeTiled_v12000 enc, cudaStream_t s, bool clear_err, bool timing) {
+  const h3blk_config& c = h->cfg;
+  const bool q = c.quant != 0;
+  const Layout L = make_layout(c, n_rows);
+  const size_t C = c.hidden, HD = (size_t)c.heads * c.head_dim, F = c.ffn;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   auto buf = [&](int stage) { return ws + L.off[stage]; };
   int* err = reinterpret_cast<int*>(buf(H3BLK_STAGE_ERROR));
@@ -286,9 +199,9 @@ int h3blk_forward(h3blk_handle h, int64_t n_rows, const void* x, const int32_t* 
     if (e_ != cudaSuccess) return H3BLK_ERR_CUDA; \
   } while (0)
 
-  auto mark = [&](int i) -> cudaError_t { return h->timing ? cudaEventRecord(h->events[i], s) : cudaSuccess; };
+  auto mark = [&](int i) -> cudaError_t { return timing ? cudaEventRecord(h->events[i], s) : cudaSuccess; };
   H3_TRY(mark(0));
-  H3_TRY(cudaMemsetAsync(err, 0, sizeof(int), s));
+  if (clear_err) H3_TRY(cudaMemsetAsync(err, 0, sizeof(int), s));
   H3_TRY(h3::launch_tile_info(tag, tidx, n_rows, c.n_tags, c.n_t, tiles, err, s));
 
   // ---- pre-attention AdaLN + RMSNorm
@@ -428,6 +341,123 @@ int h3blk_forward(h3blk_handle h, int64_t n_rows, const void* x, const int32_t* 
   return H3BLK_OK;
 }
 
+}  // namespace h3api
+
+int h3api::mod_check(const h3blk_ctx* h, const h3blk_mod_weights* w) {
+  if (!h || !w) return H3BLK_ERR_INVALID_ARG;
+  if (w->freq_dim <= 0 || w->freq_dim % 16 || w->freq_dim > 1024 || w->time_hidden <= 0 || w->time_hidden % 8 ||
+      w->time_dim <= 0 || w->time_dim % 8 || h->cfg.n_t > h3::kMaxModSets)
+    return H3BLK_ERR_UNSUPPORTED;
+  const size_t biggest = (size_t)h->cfg.n_t * (size_t)(w->time_hidden > w->time_dim ? w->time_hidden : w->time_dim);
+  if (biggest * sizeof(float) > 200 * 1024) return H3BLK_ERR_UNSUPPORTED;
+  return H3BLK_OK;
+}
+
+extern "C" {
+
+const char* h3blk_error_string(int status) {
+  switch (status) {
+    case H3BLK_OK: return "ok";
+    case H3BLK_ERR_INVALID_ARG: return "invalid argument (null or misaligned pointer, bad size, or aliasing)";
+    case H3BLK_ERR_UNSUPPORTED: return "unsupported dimension or device";
+    case H3BLK_ERR_CUDA: return "CUDA runtime or driver error";
+    case H3BLK_ERR_TIMEOUT: return "a kernel pipeline wait timed out";
+    case H3BLK_ERR_BAD_INDEX: return "a modality tag or timestep index lies outside the modulation table, or a row index outside the packed sequence";
+    default: return "unknown status";
+  }
+}
+
+int h3blk_version(void) { return kVersion; }
+
+int h3blk_create(const h3blk_config* cfg, h3blk_handle* out) {
+  if (!cfg || !out) return H3BLK_ERR_INVALID_ARG;
+  *out = nullptr;
+  const h3blk_config& c = *cfg;
+  if (c.hidden <= 0 || c.heads <= 0 || c.head_dim <= 0 || c.ffn <= 0 || c.n_tags <= 0 || c.n_t <= 0 ||
+      c.rope_pairs_t < 0 || c.rope_pairs_h < 0 || c.rope_pairs_w < 0 || !(c.rope_theta > 0.f) ||
+      !(c.norm_eps >= 0.f) || !(c.qk_norm_eps >= 0.f) || (c.quant != 0 && c.quant != 1))
+    return H3BLK_ERR_INVALID_ARG;
+  if (c.hidden % 128 || c.ffn % 128 || (c.head_dim != 64 && c.head_dim != 128) || (c.heads * c.head_dim) % 128 ||
+      c.rope_pairs_t + c.rope_pairs_h + c.rope_pairs_w > c.head_dim / 2 || c.hidden > 6144 || c.ffn > 16384 ||
+      c.heads * c.head_dim > 16384)
+    return H3BLK_ERR_UNSUPPORTED;
+  h3blk_ctx* h = new (std::nothrow) h3blk_ctx;
+  if (!h) return H3BLK_ERR_INVALID_ARG;
+  h->cfg = c;
+  h->timing = false;
+  for (auto& e : h->events) e = nullptr;
+  const int pairs[3] = {c.rope_pairs_t, c.rope_pairs_h, c.rope_pairs_w};
+  int j = 0;
+  for (int axis = 0; axis < 3; ++axis)
+    for (int i = 0; i < pairs[axis]; ++i, ++j) {
+      h->rope.axis[j] = (int8_t)axis;
+      h->rope.freq[j] = (float)std::pow((double)c.rope_theta, -(double)i / (double)pairs[axis]);
+    }
+  for (; j < h3::kMaxRopePairs; ++j) {
+    h->rope.axis[j] = 3;
+    h->rope.freq[j] = 0.f;
+  }
+  *out = h;
+  return H3BLK_OK;
+}
+
+void h3blk_destroy(h3blk_handle h) { delete h; }
+
+int h3blk_set_kernel_events(h3blk_handle h, void* const* events, int n_events) {
+  if (!h) return H3BLK_ERR_INVALID_ARG;
+  if (n_events == 0 || !events) {
+    h->timing = false;
+    return H3BLK_OK;
+  }
+  if (n_events != H3BLK_TIMING_POINTS) return H3BLK_ERR_INVALID_ARG;
+  for (int i = 0; i < n_events; ++i) {
+    if (!events[i]) return H3BLK_ERR_INVALID_ARG;
+    h->events[i] = reinterpret_cast<cudaEvent_t>(events[i]);
+  }
+  h->timing = true;
+  return H3BLK_OK;
+}
+
+int h3blk_workspace_bytes(h3blk_handle h, int64_t n_rows, size_t* bytes) {
+  if (!h || !bytes || n_rows < 1) return H3BLK_ERR_INVALID_ARG;
+  *bytes = make_layout(h->cfg, n_rows).total;
+  return H3BLK_OK;
+}
+
+int h3blk_stage_view(h3blk_handle h, int64_t n_rows, int stage, size_t* offset, size_t* bytes) {
+  if (!h || !offset || !bytes || n_rows < 1 || stage < 0 || stage >= H3BLK_STAGE_COUNT) return H3BLK_ERR_INVALID_ARG;
+  const Layout L = make_layout(h->cfg, n_rows);
+  if (L.len[stage] == 0) return H3BLK_ERR_UNSUPPORTED;  // stage not produced in this mode
+  *offset = L.off[stage];
+  *bytes = L.len[stage];
+  return H3BLK_OK;
+}
+
+int h3blk_forward(h3blk_handle h, int64_t n_rows, const void* x, const int32_t* tag, const int32_t* tidx,
+                  const int32_t* pos, const float* mod_table, const h3blk_weights* w, void* out, void* workspace,
+                  size_t workspace_bytes, void* stream) {
+  if (!h || !w || n_rows < 1 || !x || !tag || !tidx || !pos || !mod_table || !out || !workspace)
+    return H3BLK_ERR_INVALID_ARG;
+  const h3blk_config& c = h->cfg;
+  if (h3api::check_block_weights(c, w) != H3BLK_OK) return H3BLK_ERR_INVALID_ARG;
+  const void* ptrs[] = {x, tag, tidx, pos, mod_table, out, workspace};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return H3BLK_ERR_INVALID_ARG;
+  const Layout L = make_layout(c, n_rows);
+  if (workspace_bytes < L.total) return H3BLK_ERR_INVALID_ARG;
+  const size_t N = (size_t)n_rows, C = c.hidden;
+  if (overlap(out, N * C * 2, x, N * C * 2) || overlap(out, N * C * 2, workspace, L.total) ||
+      overlap(x, N * C * 2, workspace, L.total))
+    return H3BLK_ERR_INVALID_ARG;
+  int sms = 0;
+  PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+  int st = device_info(&sms, &enc);
+  if (st != H3BLK_OK) return st;
+
+  return h3api::block_forward(h, n_rows, x, tag, tidx, pos, mod_table, w, out, workspace, sms, enc,
+                              reinterpret_cast<cudaStream_t>(stream), true, h->timing);
+}
+
 int h3blk_check(h3blk_handle h, int64_t n_rows, const void* workspace, void* stream, int* status) {
   if (!h || !workspace || !status || n_rows < 1) return H3BLK_ERR_INVALID_ARG;
   const Layout L = make_layout(h->cfg, n_rows);
@@ -439,7 +469,7 @@ int h3blk_check(h3blk_handle h, int64_t n_rows, const void* workspace, void* str
     return H3BLK_ERR_CUDA;
   if (bits & (h3::kErrTimeoutGemm | h3::kErrTimeoutAttn))
     *status = H3BLK_ERR_TIMEOUT;
-  else if (bits & h3::kErrBadIndex)
+  else if (bits & (h3::kErrBadIndex | h3::kErrBadRowIndex))
     *status = H3BLK_ERR_BAD_INDEX;
   else
     *status = H3BLK_OK;
@@ -493,18 +523,9 @@ int h3blk_prepare_int8_weights(h3blk_handle h, const h3blk_weights* in, void* bl
   return H3BLK_OK;
 }
 
-static int mod_check(const h3blk_ctx* h, const h3blk_mod_weights* w) {
-  if (!h || !w) return H3BLK_ERR_INVALID_ARG;
-  if (w->freq_dim <= 0 || w->freq_dim % 16 || w->freq_dim > 1024 || w->time_hidden <= 0 || w->time_hidden % 8 ||
-      w->time_dim <= 0 || w->time_dim % 8 || h->cfg.n_t > h3::kMaxModSets)
-    return H3BLK_ERR_UNSUPPORTED;
-  const size_t biggest = (size_t)h->cfg.n_t * (size_t)(w->time_hidden > w->time_dim ? w->time_hidden : w->time_dim);
-  if (biggest * sizeof(float) > 200 * 1024) return H3BLK_ERR_UNSUPPORTED;
-  return H3BLK_OK;
-}
 
 int h3blk_modulation_scratch_bytes(h3blk_handle h, const h3blk_mod_weights* w, size_t* bytes) {
-  const int st = mod_check(h, w);
+  const int st = h3api::mod_check(h, w);
   if (st != H3BLK_OK) return st;
   if (!bytes) return H3BLK_ERR_INVALID_ARG;
   *bytes = (size_t)h->cfg.n_t * (size_t)(w->time_hidden + w->time_dim) * sizeof(float);
@@ -513,7 +534,7 @@ int h3blk_modulation_scratch_bytes(h3blk_handle h, const h3blk_mod_weights* w, s
 
 int h3blk_modulation_table(h3blk_handle h, const h3blk_mod_weights* w, const float* t_now, const float* t_end,
                            float gate, float* table, void* scratch, size_t scratch_bytes, void* stream) {
-  int st = mod_check(h, w);
+  int st = h3api::mod_check(h, w);
   if (st != H3BLK_OK) return st;
   const int V = h->cfg.n_t;
   if (!t_now || !table || !scratch || !w->w1 || !w->b1 || !w->w2 || !w->b2 || !w->adaln_w || !w->adaln_b)
@@ -532,6 +553,7 @@ int h3blk_modulation_table(h3blk_handle h, const h3blk_mod_weights* w, const flo
   h3::ModTableArgs m;
   std::memset(&m, 0, sizeof(m));
   m.n_sets = V;
+  m.n_vec = 6;
   m.n_tags = h->cfg.n_tags;
   m.hidden = h->cfg.hidden;
   m.freq_dim = w->freq_dim;

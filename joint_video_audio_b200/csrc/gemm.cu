@@ -19,6 +19,7 @@
 //   kEpiResid  out = resid + gate[tag][tidx] * acc (padding rows: out = resid).
 //   kEpiSwiGLU B holds W1 rows then W3 rows; tile j loads W1 rows j*128.. and W3
 //              rows j*128.. into its two 128-column halves: out = silu(g) * u.
+//   kEpiStoreBf16 out = acc (+ an fp32 bias per column when given).
 //   kEpiStoreS32  raw int32 accumulators (exactness tests of the int8 path).
 // int8 mode ("HyperFlow H3 Flash ...", "How it got smaller and faster":
 // rotated W8A8): kind::i8, s32 accumulators, value = acc * s_a[row] * s_b[col].
@@ -167,6 +168,16 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tacc, 
       load_chunk<INT8>(tacc + c * 32, sa, p.s_b, col, v);
       if (!row_ok) continue;
       __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + row * p.ld_out + col;
+      if (EPI == kEpiStoreBf16 && p.bias) {
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+          const float4 b4 = __ldg(reinterpret_cast<const float4*>(p.bias + col + j));
+          v[j] += b4.x;
+          v[j + 1] += b4.y;
+          v[j + 2] += b4.z;
+          v[j + 3] += b4.w;
+        }
+      }
       if (EPI == kEpiResid) {
         const uint4* rs = reinterpret_cast<const uint4*>(p.resid + row * (int64_t)p.N + col);
 #pragma unroll

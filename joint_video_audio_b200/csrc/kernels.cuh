@@ -57,7 +57,7 @@ cudaError_t launch_rotate_quant(const __nv_bfloat16* in, int64_t rows, int K, in
 
 // ---------------------------------------------------------------- GEMM
 enum GemmEpilogue : int {
-  kEpiStoreBf16 = 0,  // out = acc
+  kEpiStoreBf16 = 0,  // out = acc (+ bias[col])
   kEpiQKV = 1,        // q/k: per-head RMSNorm * gain + RoPE; v: plain
   kEpiResid = 2,      // out = resid + gate * acc
   kEpiSwiGLU = 3,     // out[:, j] = silu(acc_gate[:, j]) * acc_up[:, j]
@@ -90,6 +90,8 @@ struct GemmArgs {
   int head_dim, hd;
   float qk_eps;
   RopeTable rope;
+  // kEpiStoreBf16: optional fp32 bias added per column
+  const float* bias;
   // int8 dequantisation: acc * s_a[row] * s_b[col]
   const float* s_a;
   const float* s_b;
@@ -114,20 +116,57 @@ constexpr int kMaxModSets = 8;  // timestep sets (the table's n_t) per call
 
 struct ModTimes {
   int count;                 // 0: no embedding (the input comes from memory)
-  float t[kMaxModSets];
+  float t[kMaxModSets];      // used when dev == nullptr
+  const float* dev;          // device array of count timesteps (graph-replayable)
 };
 
 struct ModTableArgs {
   int n_sets, n_tags, hidden, freq_dim, time_hidden, time_dim;
+  int n_vec;                 // vectors per (tag, set): 6 for a block, 2 for norm_out
   ModTimes t_now, t_end;     // per set
   float gate;                // two-time blend weight of the t_end embedding
   const float *w1, *b1, *w2, *b2;
   const float *w1_r, *b1_r, *w2_r, *b2_r;
-  const __nv_bfloat16* adaln_w;  // [n_tags][6 * hidden][time_dim]
-  const float* adaln_b;          // [n_tags][6 * hidden]
-  float* table;              // [n_tags][n_sets][6 * hidden]
-  float* scratch;            // n_sets * (time_hidden + time_dim) floats
+  const __nv_bfloat16* adaln_w;  // [n_tags][n_vec * hidden][time_dim]
+  const float* adaln_b;          // [n_tags][n_vec * hidden]
+  float* table;              // [n_tags][n_sets][n_vec * hidden]
+  float* scratch;            // n_sets * (time_hidden + time_dim) floats: hidden layer, then E
 };
+// Time embedding E (into scratch + n_sets * time_hidden) and the projection.
 cudaError_t launch_modulation_table(const ModTableArgs& a, int num_sms, cudaStream_t s);
+// The two halves on their own: E = time MLP(s) of the sets' timesteps ...
+cudaError_t launch_time_embedding(const ModTableArgs& a, int num_sms, cudaStream_t s);
+// ... and table = A_tag silu(E) + a_tag from an E already in scratch.
+cudaError_t launch_adaln_projection(const ModTableArgs& a, int num_sms, cudaStream_t s);
+
+// ---------------------------------------------------------------- model shell
+// out[idx[m]] = bf16(W x[m] + b) for the M fp32 rows x [M][K]; W fp32 [C][K].
+cudaError_t launch_embed_rows(const float* x, int64_t M, int K, const float* W, const float* b, int C,
+                              const int32_t* idx, int64_t n_rows, __nv_bfloat16* out, int* err, cudaStream_t s);
+// out[idx[m]] = bf16(rmsnorm(r[m]) * gain) over C channels.
+cudaError_t launch_norm_scatter(const __nv_bfloat16* r, int64_t M, int C, const __nv_bfloat16* gain, float eps,
+                                const int32_t* idx, int64_t n_rows, __nv_bfloat16* out, int* err, cudaStream_t s);
+// y[m] = W (rmsnorm(x[idx[m]]) (1 + scale) + shift) + b, (shift, scale) =
+// table[tag][tidx][0..1] (zero for padding); W fp32 [n_out][C], y fp32.
+struct HeadArgs {
+  const __nv_bfloat16* x;
+  const int32_t* idx;
+  int64_t M, n_rows;
+  int C, n_out;
+  const int32_t* tag;
+  const int32_t* tidx;
+  const float* table;  // [n_tags][n_t][2][C]
+  int n_tags, n_t;
+  float eps;
+  const float* W;
+  const float* b;
+  float* y;
+  int* err;
+};
+cudaError_t launch_head(const HeadArgs& a, int num_sms, cudaStream_t s);
+// out_*[m] = in_*[idx[m]]
+cudaError_t launch_gather_meta(const int32_t* idx, int64_t M, int64_t n_rows, const int32_t* tag,
+                               const int32_t* tidx, const int32_t* pos, int32_t* out_tag, int32_t* out_tidx,
+                               int32_t* out_pos, int* err, cudaStream_t s);
 
 }  // namespace h3

@@ -2,7 +2,8 @@
 //
 //   e_k   = [cos(t_k w), sin(t_k w)],  w_i = 10000^(-i / (freq_dim / 2))
 //   E_k   = (1 - g) (W2 silu(W1 e(t_k) + b1) + b2) + g (W2r silu(W1r e(r_k) + b1r) + b2r)
-//   table[tag][k] = A_tag silu(E_k) + a_tag        (6 * hidden outputs)
+//   table[tag][k] = A_tag silu(E_k) + a_tag        (n_vec * hidden outputs: 6 for a
+//                                                 block, 2 for the output norm)
 //
 // Sources: "MiniMaxH3Transformer3DModel" (diffusers API page), constructor
 // (freq_dim of the sinusoidal embedding, timesteps unscaled in [0, 1]; the
@@ -67,7 +68,8 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_sets_kernel(const WT* __res
       const int v = idx / h, i = idx - v * h;
       const float w = exp2f(-(float)i / (float)h * 13.287712379549449f);  // 10000^(-i/h)
       float sn, cs;
-      sincosf(embed_t.t[v] * w, &sn, &cs);
+      const float tv = embed_t.dev ? embed_t.dev[v] : embed_t.t[v];
+      sincosf(tv * w, &sn, &cs);
       xs[v * I + i] = cs;
       xs[v * I + h + i] = sn;
     }
@@ -177,9 +179,8 @@ cudaError_t gemv(const WT* W, const float* b, int64_t wz, int64_t bz, int Z, int
 
 }  // namespace
 
-cudaError_t launch_modulation_table(const ModTableArgs& a, int num_sms, cudaStream_t s) {
+cudaError_t launch_time_embedding(const ModTableArgs& a, int num_sms, cudaStream_t s) {
   const int V = a.n_sets, F0 = a.freq_dim, Hh = a.time_hidden, Td = a.time_dim;
-  const int O = 6 * a.hidden;
   float* hid = a.scratch;                      // [V][Hh]
   float* E = a.scratch + (size_t)V * Hh;       // [V][Td]
   const ModTimes none{};
@@ -196,11 +197,22 @@ cudaError_t launch_modulation_table(const ModTableArgs& a, int num_sms, cudaStre
                     s);
     if (e != cudaSuccess) return e;
     e = gemv<float>(a.w2_r, a.b2_r, 0, 0, 1, Td, Hh, V, hid, none, false, false, g, true, E, 0, Td, num_sms, s);
-    if (e != cudaSuccess) return e;
   }
+  return e;
+}
+
+cudaError_t launch_adaln_projection(const ModTableArgs& a, int num_sms, cudaStream_t s) {
+  const int V = a.n_sets, Td = a.time_dim, O = a.n_vec * a.hidden;
+  const float* E = a.scratch + (size_t)V * a.time_hidden;
+  const ModTimes none{};
   // table[tag][k] = A_tag silu(E_k) + a_tag
   return gemv<__nv_bfloat16>(a.adaln_w, a.adaln_b, (int64_t)O * Td, O, a.n_tags, O, Td, V, E, none, true, false, 1.f,
                              false, a.table, (int64_t)V * O, O, num_sms, s);
+}
+
+cudaError_t launch_modulation_table(const ModTableArgs& a, int num_sms, cudaStream_t s) {
+  const cudaError_t e = launch_time_embedding(a, num_sms, s);
+  return e != cudaSuccess ? e : launch_adaln_projection(a, num_sms, s);
 }
 
 }  // namespace h3

@@ -14,6 +14,7 @@ enum : int {
   kErrBadIndex = 1,       // a tag or timestep index outside the modulation table
   kErrTimeoutGemm = 2,    // a GEMM pipeline wait ran out of time
   kErrTimeoutAttn = 4,    // an attention pipeline wait ran out of time
+  kErrBadRowIndex = 8,    // a row index of the model shell outside the packed sequence
 };
 
 // Wall-clock budget of a single pipeline wait before it is declared stuck.

@@ -121,22 +121,36 @@ class ModelOracle:
             parts.append((t, r))
         return scatter_rows(lay.n, d.hidden, parts)
 
-    def heads(self, x, mi, tabs):
+    def heads(self, x, mi, tabs, rows=None):
+        """Both heads. x holds every packed row, or only ``rows`` (sorted);
+        then only the video / audio rows among them are returned, with their
+        positions in video_idx / audio_idx."""
         p, lay = self.p, mi.layout
-        h = norm_out(x, tabs["out"], lay.tag, lay.tidx, p.sd.final_norm_eps)
-        return (affine(h[mi.video_idx], p.proj_out_w, p.proj_out_b),
-                affine(h[mi.audio_idx], p.audio_out_w, p.audio_out_b))
+        rows = np.arange(lay.n) if rows is None else np.asarray(rows)
+        at = {int(r): j for j, r in enumerate(rows)}
+        h = norm_out(x, tabs["out"], lay.tag[rows], lay.tidx[rows], p.sd.final_norm_eps)
+        vsel = np.array([i for i, r in enumerate(mi.video_idx) if int(r) in at], dtype=np.int64)
+        asel = np.array([i for i, r in enumerate(mi.audio_idx) if int(r) in at], dtype=np.int64)
+        hv = h[[at[int(r)] for r in mi.video_idx[vsel]]] if vsel.size else np.zeros((0, h.shape[1]))
+        ha = h[[at[int(r)] for r in mi.audio_idx[asel]]] if asel.size else np.zeros((0, h.shape[1]))
+        return (affine(hv, p.proj_out_w, p.proj_out_b), affine(ha, p.audio_out_w, p.audio_out_b), vsel, asel)
 
-    def forward(self, mi, n_layers=None):
-        """Returns dict: video, audio (velocities), x0 (packed input), x (packed
-        stack output) and the tables."""
+    def forward(self, mi, n_layers=None, rows=None):
+        """Returns dict: video, audio (velocities, for the positions
+        video_sel / audio_sel of the index tensors), x0 (packed input), x
+        (stack output, of ``rows`` only when given) and the tables. With
+        ``rows``, the last layer and the heads are evaluated for those packed
+        rows only; every earlier layer needs all rows."""
         lay = mi.layout
         tabs = self.tables(mi.t_now, mi.t_end, mi.gate)
         x0 = self.shell_in(mi, tabs)
         x = x0
         L = len(self.p.layers) if n_layers is None else n_layers
         for k in range(L):
+            sub = rows if k == L - 1 else None
             x = BlockOracle(self.d, self.p.layers[k].w).forward(x, lay.tag, lay.tidx, lay.pos,
-                                                                tabs["layers"][k])["out"]
-        v, a = self.heads(x, mi, tabs)
-        return {"video": v, "audio": a, "x0": x0, "x": x, "tables": tabs}
+                                                                tabs["layers"][k], rows=sub)["out"]
+        if rows is not None and L == 0:
+            x = x0[np.asarray(rows)]
+        v, a, vsel, asel = self.heads(x, mi, tabs, rows)
+        return {"video": v, "audio": a, "video_sel": vsel, "audio_sel": asel, "x0": x0, "x": x, "tables": tabs}

@@ -171,3 +171,118 @@ def test_modulation_producer_validation_before_gpu():
         B.H3BLK_ERR_INVALID_ARG
     assert B.h3blk_modulation_table(blk.handle, w, [0.1, 0.2], None, 0.0, 0, base, 1 << 20, None) == \
         B.H3BLK_ERR_INVALID_ARG
+
+
+# ---------------------------------------------------------------- model shell
+
+def _fake_model(n_layers=2, n_refiner=1, video_in=16, audio_in=8, text_dim=128):
+    mc = B.h3blk_model_config(n_layers=n_layers, n_refiner=n_refiner, video_in=video_in, audio_in=audio_in,
+                              text_dim=text_dim, final_norm_eps=1e-5)
+    base = 1 << 40
+    p = lambda k: base + (k << 28)  # noqa: E731  fake, 16-byte aligned device addresses
+    time = B.h3blk_mod_weights(freq_dim=64, time_hidden=128, time_dim=64, w1=p(1), b1=p(2), w2=p(3), b2=p(4))
+    blockw = lambda k: B.h3blk_weights(wqkv=p(k), q_gain=p(k + 1), k_gain=p(k + 2), wo=p(k + 3),  # noqa: E731
+                                       w13=p(k + 4), w2=p(k + 5))
+    layers = (B.h3blk_layer_weights * 2)(*[B.h3blk_layer_weights(w=blockw(20 + 10 * i), adaln_w=p(27 + 10 * i),
+                                                                 adaln_b=p(28 + 10 * i)) for i in range(2)])
+    refiner = (B.h3blk_layer_weights * 1)(B.h3blk_layer_weights(w=blockw(60), adaln_w=p(67), adaln_b=p(68)))
+    w = B.h3blk_model_weights(time=time, layers=layers, refiner=refiner, refiner_gain=p(70), out_adaln_w=p(71),
+                              out_adaln_b=p(72), proj_in_w=p(73), proj_in_b=p(74), audio_in_w=p(75),
+                              audio_in_b=p(76), ctx_w=p(77), ctx_b=p(78), proj_out_w=p(79), proj_out_b=p(80),
+                              audio_out_w=p(81), audio_out_b=p(82))
+    inp = B.h3blk_model_inputs(n_rows=320, n_video=192, n_audio=32, n_text=64, tag=p(90), tidx=p(91), pos=p(92),
+                               video_idx=p(93), audio_idx=p(94), text_idx=p(95), video=p(96), audio=p(97),
+                               text=p(98), t_now=p(99), t_end=None, gate=0.0)
+    return mc, w, inp, p
+
+
+def _model_call(blk, mc, w, inp, p, ws_bytes=None, video_out=None, audio_out=None, ws=None):
+    if ws_bytes is None:
+        ws_bytes = B.h3blk_model_workspace_bytes(blk.handle, mc, w.time, inp.n_rows, inp.n_text)
+    return B.h3blk_model_forward(blk.handle, mc, w, inp, p(100) if video_out is None else video_out,
+                                 p(101) if audio_out is None else audio_out, p(102) if ws is None else ws,
+                                 ws_bytes, None)
+
+
+def test_model_workspace_layout():
+    blk = j.H3Block(hi.TINY)
+    mc, w, inp, p = _fake_model()
+    full = B.h3blk_model_workspace_bytes(blk.handle, mc, w.time, 320, 64)
+    no_text = B.h3blk_model_workspace_bytes(blk.handle, mc, w.time, 320, 0)
+    C = hi.TINY.hidden
+    # two packed sequences and the block workspace at least; text buffers on top
+    assert no_text >= 2 * 320 * C * 2 + blk.workspace_bytes(320)
+    assert full >= no_text + 2 * 64 * C * 2
+    with pytest.raises(B.H3BlkError):
+        B.h3blk_model_workspace_bytes(blk.handle, mc, w.time, 320, 321)
+
+
+def test_model_forward_passes_validation_with_fake_pointers():
+    """A well-formed call gets through every host check and only fails at
+    the first CUDA call (no device here)."""
+    blk = j.H3Block(hi.TINY)
+    mc, w, inp, p = _fake_model()
+    assert _model_call(blk, mc, w, inp, p) == B.H3BLK_ERR_CUDA
+
+
+@pytest.mark.parametrize("case,status", [
+    ("counts_exceed_rows", B.H3BLK_ERR_INVALID_ARG),
+    ("negative_count", B.H3BLK_ERR_INVALID_ARG),
+    ("video_in_not_multiple_of_4", B.H3BLK_ERR_UNSUPPORTED),
+    ("video_in_too_wide", B.H3BLK_ERR_UNSUPPORTED),
+    ("text_dim_not_multiple_of_64", B.H3BLK_ERR_UNSUPPORTED),
+    ("null_layers", B.H3BLK_ERR_INVALID_ARG),
+    ("layer_missing_weight", B.H3BLK_ERR_INVALID_ARG),
+    ("gate_without_t_end", B.H3BLK_ERR_INVALID_ARG),
+    ("gate_out_of_range", B.H3BLK_ERR_INVALID_ARG),
+    ("workspace_too_small", B.H3BLK_ERR_INVALID_ARG),
+    ("misaligned_video", B.H3BLK_ERR_INVALID_ARG),
+    ("null_video_out", B.H3BLK_ERR_INVALID_ARG),
+    ("null_text_with_text_rows", B.H3BLK_ERR_INVALID_ARG),
+])
+def test_model_forward_rejects_bad_arguments(case, status):
+    blk = j.H3Block(hi.TINY)
+    kw = {}
+    mc_kw = {}
+    if case == "video_in_not_multiple_of_4":
+        mc_kw["video_in"] = 6
+    if case == "video_in_too_wide":
+        mc_kw["video_in"] = 132
+    if case == "text_dim_not_multiple_of_64":
+        mc_kw["text_dim"] = 100
+    mc, w, inp, p = _fake_model(**mc_kw)
+    if case == "counts_exceed_rows":
+        inp.n_text = 100
+    if case == "negative_count":
+        inp.n_audio = -1
+    if case == "null_layers":
+        w.layers = None
+    if case == "layer_missing_weight":
+        w.layers[1].w.wo = None
+    if case == "gate_without_t_end":
+        inp.gate = 0.5
+        w.time.w1_r = w.time.b1_r = w.time.w2_r = w.time.b2_r = p(5)
+    if case == "gate_out_of_range":
+        inp.gate = 1.5
+    if case == "workspace_too_small":
+        kw["ws_bytes"] = 4096
+    if case == "misaligned_video":
+        inp.video = p(96) + 4
+    if case == "null_video_out":
+        kw["video_out"] = 0
+    if case == "null_text_with_text_rows":
+        inp.text = None
+    if case in ("video_in_not_multiple_of_4", "video_in_too_wide", "text_dim_not_multiple_of_64"):
+        kw["ws_bytes"] = 1 << 40
+    assert _model_call(blk, mc, w, inp, p, **kw) == status
+
+
+def test_model_graph_create_validates_before_capture():
+    blk = j.H3Block(hi.TINY)
+    mc, w, inp, p = _fake_model()
+    inp.n_video = 400
+    with pytest.raises(B.H3BlkError) as e:
+        B.h3blk_model_graph_create(blk.handle, mc, w, inp, p(100), p(101), p(102), 1 << 40)
+    assert e.value.status == B.H3BLK_ERR_INVALID_ARG
+    assert B.h3blk_graph_launch(None, None) == B.H3BLK_ERR_INVALID_ARG
+    B.h3blk_graph_destroy(None)   # no-op

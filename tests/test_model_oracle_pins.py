@@ -184,3 +184,13 @@ def test_layer_tables_use_each_layers_projection(two_time):
     np.testing.assert_allclose(t2["layers"][1], 2 * t1["layers"][1], rtol=1e-14, atol=1e-15)
     assert t1["layers"][0].shape == (d.n_tags, d.n_t, 6, d.hidden)
     assert t1["out"].shape == (d.n_tags, d.n_t, 2, d.hidden)
+
+
+def test_subset_rows_match_the_full_forward():
+    d, p, mi = _tiny(n_layers=2)
+    full = ModelOracle(d, p).forward(mi)
+    rows = hi.sample_rows(mi.layout, k=40, k_pad=4, seed=3)
+    sub = ModelOracle(d, p).forward(mi, rows=rows)
+    np.testing.assert_allclose(sub["video"], full["video"][sub["video_sel"]], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(sub["audio"], full["audio"][sub["audio_sel"]], rtol=1e-12, atol=1e-12)
+    assert sub["video_sel"].size > 10
