@@ -404,6 +404,57 @@ def run_modulation(torch, j, hi, device, peaks, steps):
             "config": "real dims, 4 tags x 4 two-time sets, freq 256 -> 5376 -> 2688 -> 6 x 5376"}
 
 
+def run_model(torch, j, hi, device, steps, warmup, quant):
+    """The whole transformer forward (input projections, 2 token-refiner
+    blocks over the text rows, the block stack, norm_out and both heads) at real
+    dimensions on the 32k layout, replayed as one CUDA graph: 50 bf16 layers,
+    or 47 rotated-W8A8 layers with two-time conditioning. Random weights drawn
+    on the device. Also times the same graph without the stack (the shell)."""
+    from dataclasses import replace
+    if quant:
+        dims = replace(hi.REAL, n_t=4, quant=1)
+        lay = hi.layout_two_time(hi.layout_t2va_32k())
+        sd = replace(hi.REAL_SHELL, n_layers=47)
+    else:
+        dims, lay, sd = hi.REAL, hi.layout_t2va_32k(), hi.REAL_SHELL
+    params = hi.make_model_params_device(dims, hi.REAL_MOD, sd, two_time=bool(quant), device=device)
+    m = j.Model(dims, sd)
+    dm = m.load(params, device)
+    del params
+    mi = hi.make_model_inputs(dims, sd, lay, two_time=bool(quant))
+    di = j.DeviceInputs.from_model_inputs(mi, device)
+    vo, ao, ws = m.buffers(dm, di)
+    g = m.graph(dm, di, vo, ao, ws)
+    shell = j.Model(dims, replace(sd, n_layers=0))
+    g0 = shell.graph(dm, di, vo, ao, ws)
+
+    def timed(graph, n):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        for a, b in ev:
+            a.record()
+            graph.launch()
+            b.record()
+        torch.cuda.synchronize(device)
+        return [a.elapsed_time(b) for a, b in ev]
+
+    timed(g, warmup)
+    ms = statistics.mean(timed(g, steps))
+    status = j.Model.check(ws)
+    timed(g0, 3)
+    shell_ms = statistics.mean(timed(g0, 5))
+    kern, other = g.nodes
+    out = {"workload": lay.name, "layers": sd.n_layers, "refiner_layers": sd.n_refiner,
+           "mode": "w8a8" if quant else "bf16", "n_rows": lay.n, "ms_per_forward": ms,
+           "rows_per_s": lay.n / (ms / 1e3), "shell_ms": shell_ms,
+           "ms_per_layer": (ms - shell_ms) / max(1, sd.n_layers), "graph_kernels": kern,
+           "graph_other_nodes": other, "gpu_launches": kern * steps, "steps": steps, "warmup": warmup,
+           "status": status,
+           "weights_gb": round(dm.nbytes() / 1e9, 1)}
+    del g, g0, dm, di, vo, ao, ws
+    torch.cuda.empty_cache()
+    return out
+
+
 # --------------------------------------------------------------------------- CPU oracle arm
 
 def cpu_oracle_sample(name="t2va_32k", kv_rows=1024, q_rows=8, seed=0):
@@ -452,6 +503,7 @@ def main():
     ap.add_argument("--no-w8a8", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-model", action="store_true", help="skip the whole-model forward legs")
     args = ap.parse_args()
     assert args.warmup >= 3 or args.impl == "reference", "at least 3 warm-up steps"
     ws_, rank, local = dist_env()
@@ -492,6 +544,10 @@ def main():
     if not args.no_w8a8:
         w8 = run_gpu_case(torch, j, hi, "w8a8_t2va_32k", args.steps, args.warmup, device, peaks, int8_peak)
     modt = run_modulation(torch, j, hi, device, peaks, args.steps)
+    models = []
+    if not args.no_model:
+        for q in (0, 1):
+            models.append(run_model(torch, j, hi, device, min(args.steps, 3), 3, q))
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rps, secs, desc, threads = cpu_oracle_sample(args.workload)
@@ -514,6 +570,8 @@ def main():
                             "ms_per_step": w8["ms_per_step"], "roofline": w8["roofline"], "kernels": w8["kernels"],
                             "gpu_launches": w8["gpu_launches"]}
         line["modulation_table"] = modt
+        if models:
+            line["model_forward"] = models
         print(json.dumps(line), flush=True)
     import torch.distributed as dist
     if dist.is_initialized():

@@ -517,3 +517,51 @@ def make_model_inputs(dims: Dims, sd: ShellDims, layout: Layout, seed=0, two_tim
         tn = rng.uniform(0, 1, dims.n_t).astype(np.float32)
         te, gate = tn.copy(), 0.0
     return ModelInputs(layout, v, a, t, video, audio, text, tn, te, float(gate))
+
+
+def make_model_params_device(dims: Dims, md: ModDims, sd: ShellDims, seed=0, two_time=False,
+                             device="cuda") -> ModelParams:
+    """The same distributions as make_model_params, drawn on the device with a
+    seeded torch generator (not the same values): for timing full-size models
+    whose weights would take minutes to draw on the host. Block weights come
+    as h3_inputs.Weights of device tensors."""
+    g = torch.Generator(device=device)
+    g.manual_seed(seed + 80)
+    C, HD, F, D, Td = dims.hidden, dims.hd, dims.ffn, dims.head_dim, md.time_dim
+
+    def n(shape, std, dtype=torch.bfloat16, mean=0.0):
+        t = torch.randn(shape, generator=g, device=device, dtype=torch.float32 if dtype == torch.float32 else dtype)
+        t.mul_(std)
+        if mean:
+            t.add_(mean)
+        return t
+
+    def mlp():
+        return (n((md.time_hidden, md.freq_dim), 1.0 / np.sqrt(md.freq_dim), torch.float32),
+                n((md.time_hidden,), 0.02, torch.float32),
+                n((Td, md.time_hidden), 1.0 / np.sqrt(md.time_hidden), torch.float32),
+                n((Td,), 0.02, torch.float32))
+
+    def adaln(n_vec):
+        return n((dims.n_tags, n_vec * C, Td), 0.1 / np.sqrt(Td)), n((dims.n_tags, n_vec * C), 0.02, torch.float32)
+
+    def layer():
+        w = Weights(n((3 * HD, C), 1.0 / np.sqrt(C)), n((D,), 0.1, mean=1.0), n((D,), 0.1, mean=1.0),
+                    n((C, HD), 1.0 / np.sqrt(HD)), n((2 * F, C), 1.0 / np.sqrt(C)), n((C, F), 1.0 / np.sqrt(F)))
+        return Layer(w, *adaln(6))
+
+    w1, b1, w2, b2 = mlp()
+    r = mlp() if two_time else (None, None, None, None)
+    time = ModParams(md, w1, b1, w2, b2, *r, torch.zeros(1, 1, 1, dtype=torch.bfloat16, device=device),
+                     torch.zeros(1, 1, device=device))
+    layers = [layer() for _ in range(sd.n_layers)]
+    refiner = [layer() for _ in range(sd.n_refiner)]
+    oaw, oab = adaln(2)
+    f32 = torch.float32
+    return ModelParams(
+        sd, time, layers, refiner, refiner_gain=n((C,), 0.1, mean=1.0), out_adaln_w=oaw, out_adaln_b=oab,
+        proj_in_w=n((C, sd.video_in), 1.0 / np.sqrt(sd.video_in), f32), proj_in_b=n((C,), 0.02, f32),
+        audio_in_w=n((C, sd.audio_in), 1.0 / np.sqrt(sd.audio_in), f32), audio_in_b=n((C,), 0.02, f32),
+        ctx_w=n((C, sd.text_dim), 1.0 / np.sqrt(sd.text_dim)), ctx_b=n((C,), 0.02, f32),
+        proj_out_w=n((sd.video_in, C), 1.0 / np.sqrt(C), f32), proj_out_b=n((sd.video_in,), 0.02, f32),
+        audio_out_w=n((sd.audio_in, C), 1.0 / np.sqrt(C), f32), audio_out_b=n((sd.audio_in,), 0.02, f32))

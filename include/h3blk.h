@@ -348,6 +348,9 @@ H3BLK_API int h3blk_model_graph_create(h3blk_handle h, const h3blk_model_config*
                                        const h3blk_model_inputs* in, float* video_out, float* audio_out,
                                        void* workspace, size_t workspace_bytes, h3blk_graph* out);
 H3BLK_API int h3blk_graph_launch(h3blk_graph g, void* stream);
+/* Node census of the captured forward: kernel launches (every one of them a
+ * kernel of this library) and other nodes (memsets). */
+H3BLK_API int h3blk_graph_info(h3blk_graph g, int* kernel_nodes, int* other_nodes);
 H3BLK_API void h3blk_graph_destroy(h3blk_graph g);
 
 /* Document-masked attention of the block (the same kernels as the attention

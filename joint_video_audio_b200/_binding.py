@@ -29,7 +29,7 @@ EXPORTS = ["h3blk_create", "h3blk_destroy", "h3blk_workspace_bytes", "h3blk_stag
            "h3blk_gemm_s8_s32", "h3blk_gemm_bf16", "h3blk_error_string", "h3blk_version",
            "h3blk_set_kernel_events", "h3blk_attention_noalloc", "h3blk_modulation_scratch_bytes",
            "h3blk_modulation_table", "h3blk_model_workspace_bytes", "h3blk_model_forward", "h3blk_model_check",
-           "h3blk_model_graph_create", "h3blk_graph_launch", "h3blk_graph_destroy"]
+           "h3blk_model_graph_create", "h3blk_graph_launch", "h3blk_graph_info", "h3blk_graph_destroy"]
 
 H3BLK_TIMING_POINTS = 11
 TIMING_INTERVALS = ["prep", "norm1", "qkv_gemm", "attention", "quant_o", "out_proj_gemm", "norm2",
@@ -122,6 +122,7 @@ def _load():
         "h3blk_model_graph_create": (i32, [vp, C.POINTER(h3blk_model_config), C.POINTER(h3blk_model_weights),
                                             C.POINTER(h3blk_model_inputs), vp, vp, vp, sz, C.POINTER(vp)]),
         "h3blk_graph_launch": (i32, [vp, vp]),
+        "h3blk_graph_info": (i32, [vp, C.POINTER(i32), C.POINTER(i32)]),
         "h3blk_graph_destroy": (None, [vp]),
     }
     for name, (res, args) in sig.items():
@@ -282,6 +283,12 @@ def h3blk_model_graph_create(handle, mc, w, inp, video_out, audio_out, workspace
 
 def h3blk_graph_launch(graph, stream) -> int:
     return _lib.h3blk_graph_launch(graph, stream)
+
+
+def h3blk_graph_info(graph) -> tuple[int, int]:
+    k, o = C.c_int(), C.c_int()
+    _check("h3blk_graph_info", _lib.h3blk_graph_info(graph, C.byref(k), C.byref(o)))
+    return k.value, o.value
 
 
 def h3blk_graph_destroy(graph) -> None:

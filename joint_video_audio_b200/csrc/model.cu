@@ -267,6 +267,7 @@ int run_forward(const h3blk_ctx* h, const h3blk_model_config* mc, const h3blk_mo
 
 struct h3blk_graph_s {
   cudaGraphExec_t exec;
+  int kernel_nodes, other_nodes;
 };
 
 extern "C" {
@@ -329,6 +330,23 @@ int h3blk_model_graph_create(h3blk_handle h, const h3blk_model_config* mc, const
     cudaGetLastError();
     return st != H3BLK_OK ? st : H3BLK_ERR_CUDA;
   }
+  // node census: kernel launches vs memsets and the like
+  int kernels = 0, others = 0;
+  size_t n_nodes = 0;
+  if (cudaGraphGetNodes(graph, nullptr, &n_nodes) == cudaSuccess && n_nodes > 0) {
+    cudaGraphNode_t* nodes = new (std::nothrow) cudaGraphNode_t[n_nodes];
+    if (nodes && cudaGraphGetNodes(graph, nodes, &n_nodes) == cudaSuccess) {
+      for (size_t i = 0; i < n_nodes; ++i) {
+        cudaGraphNodeType t;
+        if (cudaGraphNodeGetType(nodes[i], &t) != cudaSuccess) continue;
+        if (t == cudaGraphNodeTypeKernel)
+          ++kernels;
+        else
+          ++others;
+      }
+    }
+    delete[] nodes;
+  }
   cudaGraphExec_t exec = nullptr;
   const cudaError_t e_inst = cudaGraphInstantiate(&exec, graph, 0);
   cudaGraphDestroy(graph);
@@ -339,6 +357,8 @@ int h3blk_model_graph_create(h3blk_handle h, const h3blk_model_config* mc, const
     return H3BLK_ERR_INVALID_ARG;
   }
   g->exec = exec;
+  g->kernel_nodes = kernels;
+  g->other_nodes = others;
   *out = g;
   return H3BLK_OK;
 }
@@ -346,6 +366,13 @@ int h3blk_model_graph_create(h3blk_handle h, const h3blk_model_config* mc, const
 int h3blk_graph_launch(h3blk_graph g, void* stream) {
   if (!g) return H3BLK_ERR_INVALID_ARG;
   return h3api::cuda_status(cudaGraphLaunch(g->exec, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int h3blk_graph_info(h3blk_graph g, int* kernel_nodes, int* other_nodes) {
+  if (!g || !kernel_nodes || !other_nodes) return H3BLK_ERR_INVALID_ARG;
+  *kernel_nodes = g->kernel_nodes;
+  *other_nodes = g->other_nodes;
+  return H3BLK_OK;
 }
 
 void h3blk_graph_destroy(h3blk_graph g) {

@@ -46,6 +46,16 @@ class DeviceModel:
         self.c = B.h3blk_model_weights(time=self.time.c, layers=self._layers, refiner=self._refiner,
                                        **{k: v.data_ptr() for k, v in self.t.items()})
 
+    def nbytes(self) -> int:
+        """Device bytes of every weight this model holds."""
+        ts = list(self.t.values()) + list(self.time.t.values())
+        for k in self._keep:
+            if isinstance(k, DeviceWeights):
+                ts += list(k.t.values()) + ([k.blob] if getattr(k, "blob", None) is not None else [])
+            else:
+                ts.append(k)
+        return sum(t.numel() * t.element_size() for t in ts if t is not None)
+
 
 class DeviceInputs:
     """One packed sequence's inputs on the GPU (int32 indices, fp32 latents,
@@ -129,6 +139,11 @@ class ModelGraph:
     def __init__(self, handle, keepalive):
         self.handle = handle
         self._keep = keepalive
+
+    @property
+    def nodes(self) -> tuple[int, int]:
+        """(kernel launches, other nodes) of one replay."""
+        return B.h3blk_graph_info(self.handle)
 
     def launch(self):
         st = B.h3blk_graph_launch(self.handle, _stream())
