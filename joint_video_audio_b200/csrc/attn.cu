@@ -19,8 +19,10 @@
 //   warps 2..5  softmax of query tile 0, warps 6..9 of query tile 1; one
 //               thread per query row: S row from TMEM, mask, online max / sum
 //               in the exp2 domain, P packed to bf16 pairs and stored back
-//               into the first 64 columns of its own S in TMEM, and the rescale
-//               of O in TMEM when the running max grows by more than 2^8
+//               into the first 64 columns of its own S in TMEM (each half of
+//               P announced on its own barrier, so P V starts on keys 0..63
+//               while keys 64..127 are exponentiated), and the rescale of O
+//               in TMEM when the running max grows by more than 2^8
 //               (otherwise the stale max is kept, so P stays below 256).
 // The P V product reads P straight from tensor memory (A operand in TMEM, V
 // from shared memory), so P never touches shared memory: the shared-memory
@@ -59,7 +61,7 @@ struct AttnSmem {
   static constexpr int kRegion = kTile * 128;       // 128 rows x 128 bytes (one swizzle region)
   static constexpr size_t kBytes = 1024 + 2 * (size_t)kQBytes + kSlots * (size_t)kKVBytes + 512;
   uint8_t *q0, *slot0;  // query tile t at q0 + t * kQBytes, ring slot i at slot0 + i * kKVBytes
-  uint64_t *q_full, *ring_full, *ring_empty, *s_full, *p_full, *o_final;
+  uint64_t *q_full, *ring_full, *ring_empty, *s_full, *p_lo, *p_hi, *o_final;
   uint32_t* tmem_base;
   int* abort;
 
@@ -75,10 +77,11 @@ struct AttnSmem {
     ring_full = b + 1;
     ring_empty = b + 1 + kSlots;
     s_full = b + 1 + 2 * kSlots;
-    p_full = s_full + 2;
-    o_final = s_full + 4;
-    tmem_base = reinterpret_cast<uint32_t*>(s_full + 5);
-    abort = reinterpret_cast<int*>(s_full + 6);
+    p_lo = s_full + 2;
+    p_hi = s_full + 4;
+    o_final = s_full + 6;
+    tmem_base = reinterpret_cast<uint32_t*>(s_full + 7);
+    abort = reinterpret_cast<int*>(s_full + 8);
   }
 };
 
@@ -138,7 +141,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s.s_full[i], 1);
-      mbar_init(&s.p_full[i], 4);
+      mbar_init(&s.p_lo[i], 4);
+      mbar_init(&s.p_hi[i], 4);
     }
     mbar_init(s.o_final, 1);
     *s.abort = 0;
@@ -171,7 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         bool ok = true;
         for (int kv = 0; kv < 2; ++kv, ++u) {  // K_j then V_j
           const int sl = u % kSlots;
-          if (!mbar_wait(&s.ring_empty[sl], ((u / kSlots) & 1) ^ 1, abort)) {
+          if (!mbar_wait_relaxed(&s.ring_empty[sl], ((u / kSlots) & 1) ^ 1, abort)) {
             fail(p.err, abort);
             ok = false;
             break;
@@ -214,14 +218,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       };
       // O_t += P_t V_j into TMEM columns [256 + t*128, ...); P_t is read from
       // TMEM columns [t*128, t*128 + 64), 8 columns per K = 16 step
+      // Each half of P (keys 0..63, 64..127) has its own ready barrier, so the
+      // first four K steps run while the softmax still works on the second half.
       auto issue_pv = [&](int t, int j) -> bool {
-        if (!mbar_wait(&s.p_full[t], j & 1, abort)) return false;
-        tc_fence_after();
         const uint32_t va = ring0 + slot_of(2 * j + 1) * SM::kKVBytes;
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk) {
-          const uint64_t bd = sw128_desc(va + kk * 16 * 128, SM::kRegion);
-          mma_bf16_ts(tmem + 256 + t * kTile, tmem + t * kTile + kk * 8, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+        for (int half = 0; half < 2; ++half) {
+          if (!mbar_wait(half == 0 ? &s.p_lo[t] : &s.p_hi[t], j & 1, abort)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 4 * half; kk < 4 * half + 4; ++kk) {
+            const uint64_t bd = sw128_desc(va + kk * 16 * 128, SM::kRegion);
+            mma_bf16_ts(tmem + 256 + t * kTile, tmem + t * kTile + kk * 8, bd, idesc_pv,
+                        (j > 0 || kk > 0) ? 1u : 0u);
+          }
         }
         return true;
       };
@@ -230,10 +240,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         ok = wait_ring(0) && issue_s(0, 0) && issue_s(1, 0);
         if (ok) mma_commit(&s.ring_empty[slot_of(0)]);
         for (int j = 0; ok && j < n_kv; ++j) {
-          ok = wait_ring(2 * j + 1) && issue_pv(0, j);
-          if (!ok) break;
+          // the ring waits come first: they are normally satisfied long before
+          // P, and polling them between P V and the next S would put their
+          // latency on the critical path
           const bool more = j + 1 < n_kv;
-          if (more) ok = wait_ring(2 * j + 2) && issue_s(0, j + 1);
+          ok = wait_ring(2 * j + 1) && (!more || wait_ring(2 * j + 2)) && issue_pv(0, j);
+          if (!ok) break;
+          if (more) ok = issue_s(0, j + 1);
           if (!ok) break;
           ok = issue_pv(1, j);
           if (!ok) break;
@@ -266,8 +279,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     float m_run = -CUDART_INF_F, l_run = 0.f;
     bool ok = true;
     int j = 0;
-    for (int kt = next_kv_tile(p.tiles, n_tiles, qk0, qk1, 0); kt < n_tiles;
-         kt = next_kv_tile(p.tiles, n_tiles, qk0, qk1, kt + 1), ++j) {
+    int kt = next_kv_tile(p.tiles, n_tiles, qk0, qk1, 0);
+    TileInfo ti_next;
+    if (kt < n_tiles) ti_next = p.tiles[kt];
+    for (; kt < n_tiles; ++j) {
+      const TileInfo ti = ti_next;
+      // the next KV tile's summary is fetched before waiting for S, so its
+      // global-memory latency hides behind the wait
+      const int kt_next = next_kv_tile(p.tiles, n_tiles, qk0, qk1, kt + 1);
+      if (kt_next < n_tiles) ti_next = p.tiles[kt_next];
       if (!mbar_wait(&s.s_full[t], j & 1, abort)) {
         ok = false;
         break;
@@ -277,7 +297,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       tmem_ld128(t_s, u);
       float* sv = reinterpret_cast<float*>(u);
       {
-        const TileInfo& ti = p.tiles[kt];
         const int kk = tile_kind(ti);
         if (!(kk == myk && myk != 2) || ti.rows < kTile) {
           const int rows = ti.rows;
@@ -307,11 +326,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       // exponentials on pairs: x = s * scale - m with one packed FMA; one pair
       // in kPolyEvery goes through the FMA-pipe polynomial, the rest through
       // the MUFU, so both units share the load. P is packed to bf16 pairs in
-      // place (u[0..63]); the row sum runs in two packed accumulators.
+      // place (u[0..63]); the row sum runs in two packed accumulators. Each
+      // half of P (keys 0..63, then 64..127) is stored and announced on its
+      // own barrier, so the P V product starts on the first half while the
+      // second is computed.
       const uint64_t sc2 = f2_pack(scale_log2, scale_log2), nm2 = f2_pack(-m_sub, -m_sub);
       uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = acc0;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {  // two halves of 64 columns -> 32 packed words each
+      for (int h = 0; h < 2; ++h) {
 #pragma unroll
         for (int c = 64 * h; c < 64 * h + 64; c += 2) {
           float x0, x1;
@@ -331,27 +353,29 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         }
         // P half -> tensor memory, over the first 64 columns of this tile's S
         tmem_st32(t_s + 32 * h, *reinterpret_cast<const uint32_t(*)[32]>(u + 32 * h));
+        if (h == 0 && j > 0 && __any_sync(0xffffffffu, grow)) {
+          // O must be rescaled before the first P V step of this tile adds to
+          // it; S_t of this tile completing implied the previous P V completed
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(t_o + c * 32, o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(t_o + c * 32, o);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(h == 0 ? &s.p_lo[t] : &s.p_hi[t]);
       }
       float rs0, rs1;
       f2_unpack(f2_add(acc0, acc1), rs0, rs1);
-      if (j > 0 && __any_sync(0xffffffffu, grow)) {
-        tc_fence_after();
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(t_o + c * 32, o);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(t_o + c * 32, o);
-        }
-        tmem_wait_st();
-      }
       l_run = l_run * alpha + (rs0 + rs1);
       m_run = m_use;
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s.p_full[t]);
+      kt = kt_next;
     }
     if (!ok) {
       if (lane == 0) fail(p.err, abort);
