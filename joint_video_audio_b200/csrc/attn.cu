@@ -309,16 +309,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
           }
         }
       }
-      // row max: four independent chains of three-input max
-      float m4a = -CUDART_INF_F, m4b = -CUDART_INF_F, m4c = -CUDART_INF_F, m4d = -CUDART_INF_F;
+      // row max: eight independent chains of three-input max
+      float mc[8];
 #pragma unroll
-      for (int c = 0; c < kTile; c += 8) {
-        m4a = max3f(m4a, sv[c], sv[c + 1]);
-        m4b = max3f(m4b, sv[c + 2], sv[c + 3]);
-        m4c = max3f(m4c, sv[c + 4], sv[c + 5]);
-        m4d = max3f(m4d, sv[c + 6], sv[c + 7]);
-      }
-      const float m_new = fmaxf(m_run, fmaxf(fmaxf(m4a, m4b), fmaxf(m4c, m4d)) * scale_log2);
+      for (int i = 0; i < 8; ++i) mc[i] = fmaxf(sv[2 * i], sv[2 * i + 1]);
+#pragma unroll
+      for (int c = 16; c < kTile; c += 16)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mc[i] = max3f(mc[i], sv[c + 2 * i], sv[c + 2 * i + 1]);
+      const float m8 = fmaxf(max3f(mc[0], mc[1], mc[2]), max3f(mc[3], mc[4], max3f(mc[5], mc[6], mc[7])));
+      const float m_new = fmaxf(m_run, m8 * scale_log2);
       const bool grow = m_new > m_run + kRescaleThreshold || (m_run == -CUDART_INF_F && m_new != -CUDART_INF_F);
       const float m_use = grow ? m_new : m_run;
       const float m_sub = m_use == -CUDART_INF_F ? 0.f : m_use;
