@@ -333,8 +333,8 @@ H3BLK_API int h3blk_model_forward(h3blk_handle h, const h3blk_model_config* mc, 
                                   const h3blk_model_inputs* in, float* video_out, float* audio_out, void* workspace,
                                   size_t workspace_bytes, void* stream);
 
-/* Synchronises `stream`, then reads the error word a model forward left in
- * `workspace` (sticky over all its layers). */
+/* Synchronises `stream`, then reads the error word a model forward (sticky
+ * over all its layers) or a sequence-parallel phase left in `workspace`. */
 H3BLK_API int h3blk_model_check(const void* workspace, void* stream, int* status);
 
 /* CUDA graph of one model forward: the same launches as h3blk_model_forward,
@@ -352,6 +352,51 @@ H3BLK_API int h3blk_graph_launch(h3blk_graph g, void* stream);
  * kernel of this library) and other nodes (memsets). */
 H3BLK_API int h3blk_graph_info(h3blk_graph g, int* kernel_nodes, int* other_nodes);
 H3BLK_API void h3blk_graph_destroy(h3blk_graph g);
+
+/* ------------------------------------------- sequence parallelism (Ulysses) */
+/* One block forward split over a group of `world` ranks ("HyperFlow for
+ * MiniMax-H3" model card: summary table, Usage and Performance, Ulysses
+ * context parallelism over up to four GPUs). Rank r holds the contiguous rows
+ * [r * N/world, (r+1) * N/world) of the packed sequence; attention, the one
+ * step that needs every row, runs head-parallel: rank r computes heads
+ * [r * H/world, (r+1) * H/world) over all N rows.
+ *
+ * The row -> head-group exchange is fused into the QKV projection (each head's
+ * q / k / v is stored straight into qkv[owner of its head group]) and the
+ * head-group -> row exchange into the attention epilogue (each output row is
+ * stored straight into o[owner of the row]). The pointers are peer memory
+ * (another GPU's buffer mapped into this process) or, for a collective-based
+ * exchange, this rank's own send buffers.
+ *
+ * Three calls per block, ordered across the group by the caller: every rank's
+ * h3blk_ulysses_qkv before any rank's h3blk_ulysses_attention, and every
+ * rank's attention before any rank's h3blk_ulysses_out (one stream on one
+ * device, or a group barrier between the phases). Per rank:
+ *   qkv  bf16 [N][3 * H/world * head_dim]  (q heads | k heads | v heads of its group)
+ *   o    bf16 [N/world][H * head_dim]
+ * tag, tidx, pos cover the whole sequence ([N], [N], [N][3]); x, out, and
+ * the workspace are the rank's own. UNSUPPORTED unless world divides both H
+ * and N; world <= H3BLK_MAX_RANKS. Errors are read with h3blk_model_check
+ * on the workspace. */
+#define H3BLK_MAX_RANKS 8
+typedef struct {
+  int world;
+  int rank;
+  void* qkv[H3BLK_MAX_RANKS];  /* every rank's head-group buffer */
+  void* o[H3BLK_MAX_RANKS];    /* every rank's attention-output buffer */
+} h3blk_ulysses;
+H3BLK_API int h3blk_ulysses_buffer_bytes(h3blk_handle h, int64_t n_rows, int world, size_t* qkv_bytes,
+                                         size_t* o_bytes);
+H3BLK_API int h3blk_ulysses_workspace_bytes(h3blk_handle h, int64_t n_rows, int world, size_t* bytes);
+H3BLK_API int h3blk_ulysses_qkv(h3blk_handle h, int64_t n_rows, const h3blk_ulysses* u, const void* x_local,
+                                const int32_t* tag, const int32_t* tidx, const int32_t* pos, const float* mod_table,
+                                const h3blk_weights* w, void* workspace, size_t workspace_bytes, void* stream);
+H3BLK_API int h3blk_ulysses_attention(h3blk_handle h, int64_t n_rows, const h3blk_ulysses* u, const int32_t* tag,
+                                      void* workspace, size_t workspace_bytes, void* stream);
+H3BLK_API int h3blk_ulysses_out(h3blk_handle h, int64_t n_rows, const h3blk_ulysses* u, const void* x_local,
+                                const int32_t* tag, const int32_t* tidx, const float* mod_table,
+                                const h3blk_weights* w, void* out_local, void* workspace, size_t workspace_bytes,
+                                void* stream);
 
 /* Document-masked attention of the block (the same kernels as the attention
  * step of h3blk_forward) for callers that cannot allocate device memory at run

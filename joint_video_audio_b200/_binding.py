@@ -29,7 +29,11 @@ EXPORTS = ["h3blk_create", "h3blk_destroy", "h3blk_workspace_bytes", "h3blk_stag
            "h3blk_gemm_s8_s32", "h3blk_gemm_bf16", "h3blk_error_string", "h3blk_version",
            "h3blk_set_kernel_events", "h3blk_attention_noalloc", "h3blk_modulation_scratch_bytes",
            "h3blk_modulation_table", "h3blk_model_workspace_bytes", "h3blk_model_forward", "h3blk_model_check",
-           "h3blk_model_graph_create", "h3blk_graph_launch", "h3blk_graph_info", "h3blk_graph_destroy"]
+           "h3blk_model_graph_create", "h3blk_graph_launch", "h3blk_graph_info", "h3blk_graph_destroy",
+           "h3blk_ulysses_buffer_bytes", "h3blk_ulysses_workspace_bytes", "h3blk_ulysses_qkv",
+           "h3blk_ulysses_attention", "h3blk_ulysses_out"]
+
+H3BLK_MAX_RANKS = 8
 
 H3BLK_TIMING_POINTS = 11
 TIMING_INTERVALS = ["prep", "norm1", "qkv_gemm", "attention", "quant_o", "out_proj_gemm", "norm2",
@@ -84,6 +88,10 @@ class h3blk_model_inputs(C.Structure):
                 ("t_now", C.c_void_p), ("t_end", C.c_void_p), ("gate", C.c_float)]
 
 
+class h3blk_ulysses(C.Structure):
+    _fields_ = [("world", C.c_int), ("rank", C.c_int), ("qkv", C.c_void_p * 8), ("o", C.c_void_p * 8)]
+
+
 class H3BlkError(RuntimeError):
     def __init__(self, fn, status):
         super().__init__(f"{fn} failed: status {status} ({error_string(status)})")
@@ -124,6 +132,13 @@ def _load():
         "h3blk_graph_launch": (i32, [vp, vp]),
         "h3blk_graph_info": (i32, [vp, C.POINTER(i32), C.POINTER(i32)]),
         "h3blk_graph_destroy": (None, [vp]),
+        "h3blk_ulysses_buffer_bytes": (i32, [vp, i64, i32, C.POINTER(sz), C.POINTER(sz)]),
+        "h3blk_ulysses_workspace_bytes": (i32, [vp, i64, i32, C.POINTER(sz)]),
+        "h3blk_ulysses_qkv": (i32, [vp, i64, C.POINTER(h3blk_ulysses), vp, vp, vp, vp, vp, C.POINTER(h3blk_weights),
+                                    vp, sz, vp]),
+        "h3blk_ulysses_attention": (i32, [vp, i64, C.POINTER(h3blk_ulysses), vp, vp, sz, vp]),
+        "h3blk_ulysses_out": (i32, [vp, i64, C.POINTER(h3blk_ulysses), vp, vp, vp, vp, C.POINTER(h3blk_weights), vp,
+                                    vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -293,3 +308,30 @@ def h3blk_graph_info(graph) -> tuple[int, int]:
 
 def h3blk_graph_destroy(graph) -> None:
     _lib.h3blk_graph_destroy(graph)
+
+
+def h3blk_ulysses_buffer_bytes(handle, n_rows, world) -> tuple[int, int]:
+    q, o = C.c_size_t(), C.c_size_t()
+    _check("h3blk_ulysses_buffer_bytes", _lib.h3blk_ulysses_buffer_bytes(handle, n_rows, world, C.byref(q), C.byref(o)))
+    return q.value, o.value
+
+
+def h3blk_ulysses_workspace_bytes(handle, n_rows, world) -> int:
+    n = C.c_size_t()
+    _check("h3blk_ulysses_workspace_bytes", _lib.h3blk_ulysses_workspace_bytes(handle, n_rows, world, C.byref(n)))
+    return n.value
+
+
+def h3blk_ulysses_qkv(handle, n_rows, u, x_local, tag, tidx, pos, table, w, workspace, workspace_bytes, stream) -> int:
+    return _lib.h3blk_ulysses_qkv(handle, n_rows, C.byref(u), x_local, tag, tidx, pos, table, C.byref(w), workspace,
+                                  workspace_bytes, stream)
+
+
+def h3blk_ulysses_attention(handle, n_rows, u, tag, workspace, workspace_bytes, stream) -> int:
+    return _lib.h3blk_ulysses_attention(handle, n_rows, C.byref(u), tag, workspace, workspace_bytes, stream)
+
+
+def h3blk_ulysses_out(handle, n_rows, u, x_local, tag, tidx, table, w, out_local, workspace, workspace_bytes,
+                      stream) -> int:
+    return _lib.h3blk_ulysses_out(handle, n_rows, C.byref(u), x_local, tag, tidx, table, C.byref(w), out_local,
+                                  workspace, workspace_bytes, stream)

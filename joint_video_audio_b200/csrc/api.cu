@@ -176,169 +176,227 @@ int check_block_weights(const h3blk_config& c, const h3blk_weights* w) {
 
 size_t block_workspace_bytes(const h3blk_config& c, int64_t n) { return make_layout(c, n).total; }
 
-int block_forward(const h3blk_ctx* h, int64_t n_rows, const void* x, const int32_t* tag, const int32_t* tidx,
-                  const int32_t* pos, const float* mod_table, const h3blk_weights* w, void* out, void* workspace,
-                  int sms, PFN_cuTensorMapEncodeTiled_v12000 enc, cudaStream_t s, bool clear_err, bool timing) {
-  const h3blk_config& c = h->cfg;
-  const bool q = c.quant != 0;
-  const Layout L = make_layout(c, n_rows);
-  const size_t C = c.hidden, HD = (size_t)c.heads * c.head_dim, F = c.ffn;
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  auto buf = [&](int stage) { return ws + L.off[stage]; };
-  int* err = reinterpret_cast<int*>(buf(H3BLK_STAGE_ERROR));
-  h3::TileInfo* tiles = reinterpret_cast<h3::TileInfo*>(ws + L.tiles_off);
-  auto* xb = static_cast<const __nv_bfloat16*>(x);
-  auto* qkv = reinterpret_cast<__nv_bfloat16*>(buf(H3BLK_STAGE_QKV));
-  auto* o = reinterpret_cast<__nv_bfloat16*>(buf(H3BLK_STAGE_O));
-  auto* x1 = reinterpret_cast<__nv_bfloat16*>(buf(H3BLK_STAGE_X1));
-  auto* a = reinterpret_cast<__nv_bfloat16*>(buf(H3BLK_STAGE_A));
-
-#define H3_TRY(expr)                       \
-  do {                                     \
-    cudaError_t e_ = (expr);               \
+#define H3_TRY(expr)                              \
+  do {                                            \
+    cudaError_t e_ = (expr);                      \
     if (e_ != cudaSuccess) return H3BLK_ERR_CUDA; \
   } while (0)
 
-  auto mark = [&](int i) -> cudaError_t { return timing ? cudaEventRecord(h->events[i], s) : cudaSuccess; };
-  H3_TRY(mark(0));
-  if (clear_err) H3_TRY(cudaMemsetAsync(err, 0, sizeof(int), s));
-  H3_TRY(h3::launch_tile_info(tag, tidx, n_rows, c.n_tags, c.n_t, tiles, err, s));
+namespace {
+cudaError_t mark(const h3blk_ctx* h, bool timing, int i, cudaStream_t s) {
+  return timing ? cudaEventRecord(h->events[i], s) : cudaSuccess;
+}
+}  // namespace
 
-  // ---- pre-attention AdaLN + RMSNorm
+int phase_qkv(const h3blk_ctx* h, const Span& sp, const void* x, const int32_t* tag, const int32_t* tidx,
+              const int32_t* pos, const float* mod_table, const h3blk_weights* w, const BlockBufs& b,
+              const QkvRoute* route, int sms, PFN_cuTensorMapEncodeTiled_v12000 enc, cudaStream_t s, bool clear_err,
+              bool timing) {
+  const h3blk_config& c = h->cfg;
+  const bool q = c.quant != 0;
+  const size_t HD = (size_t)c.heads * c.head_dim;
+  H3_TRY(mark(h, timing, 0, s));
+  if (clear_err) H3_TRY(cudaMemsetAsync(b.err, 0, sizeof(int), s));
+  // the tile summary covers the whole sequence: attention reads every row
+  H3_TRY(h3::launch_tile_info(tag, tidx, sp.n_total, c.n_tags, c.n_t, b.tiles, b.err, s));
+
+  // ---- pre-attention AdaLN + RMSNorm of this call's rows
   h3::ModNormArgs mn;
   std::memset(&mn, 0, sizeof(mn));
-  mn.x = xb;
-  mn.tag = tag;
-  mn.tidx = tidx;
+  mn.x = static_cast<const __nv_bfloat16*>(x);
+  mn.tag = tag + sp.row0;
+  mn.tidx = tidx + sp.row0;
   mn.table = mod_table;
-  mn.n = n_rows;
+  mn.n = sp.n_local;
   mn.C = c.hidden;
   mn.n_tags = c.n_tags;
   mn.n_t = c.n_t;
   mn.shift_idx = 0;
   mn.scale_idx = 1;
   mn.eps = c.norm_eps;
-  if (q) {
-    mn.out_q = reinterpret_cast<int8_t*>(buf(H3BLK_STAGE_H1_Q8));
-    mn.out_scale = reinterpret_cast<float*>(buf(H3BLK_STAGE_H1_SCALE));
-  } else {
-    mn.out_bf16 = reinterpret_cast<__nv_bfloat16*>(buf(H3BLK_STAGE_H1));
-  }
-  H3_TRY(mark(1));
+  mn.out_q = b.h1_q;
+  mn.out_scale = b.h1_s;
+  mn.out_bf16 = b.h1;
+  if (q) mn.out_bf16 = nullptr;
+  H3_TRY(mark(h, timing, 1, s));
   H3_TRY(h3::launch_modnorm(mn, s));
 
-  // ---- QKV projection + QK-RMSNorm + RoPE
-  GemmArgs g = base_gemm(h, err);
-  g.A = q ? (const void*)buf(H3BLK_STAGE_H1_Q8) : (const void*)buf(H3BLK_STAGE_H1);
+  // ---- QKV projection + QK-RMSNorm + RoPE (optionally routed by head group)
+  GemmArgs g = base_gemm(h, b.err);
+  g.A = q ? (const void*)b.h1_q : (const void*)b.h1;
   g.B = w->wqkv;
-  g.M = n_rows;
+  g.M = sp.n_local;
   g.N = (int)(3 * HD);
   g.Nb = (int)(3 * HD);
   g.K = c.hidden;
   g.epi = h3::kEpiQKV;
-  g.out = qkv;
+  g.out = b.qkv;
   g.ld_out = 3 * HD;
   g.q_gain = static_cast<const __nv_bfloat16*>(w->q_gain);
   g.k_gain = static_cast<const __nv_bfloat16*>(w->k_gain);
-  g.pos = pos;
-  g.s_a = q ? reinterpret_cast<const float*>(buf(H3BLK_STAGE_H1_SCALE)) : nullptr;
+  g.pos = pos + 3 * sp.row0;
+  g.s_a = q ? b.h1_s : nullptr;
   g.s_b = w->s_qkv;
-  H3_TRY(mark(2));
+  if (route) {
+    g.route_ranks = route->ranks;
+    g.route_hg = route->hg;
+    g.route_row0 = sp.row0;
+    for (int r = 0; r < route->ranks; ++r) g.route_dst[r] = route->dst[r];
+  }
+  H3_TRY(mark(h, timing, 2, s));
   H3_TRY(h3::launch_gemm(g, enc, sms, s));
+  return H3BLK_OK;
+}
 
-  // ---- attention
+int phase_attention(const h3blk_ctx* h, int64_t n_total, int heads, const int32_t* tag, const BlockBufs& b,
+                    const ORoute* route, PFN_cuTensorMapEncodeTiled_v12000 enc, cudaStream_t s, bool timing) {
   h3::AttnArgs at;
-  at.qkv = qkv;
-  at.o = o;
+  std::memset(&at, 0, sizeof(at));
+  at.qkv = b.qkv;
+  at.o = b.o;
   at.tag = tag;
-  at.tiles = tiles;
-  at.n = n_rows;
-  at.heads = c.heads;
-  at.head_dim = c.head_dim;
-  at.err = err;
-  H3_TRY(mark(3));
+  at.tiles = b.tiles;
+  at.n = n_total;
+  at.heads = heads;
+  at.head_dim = h->cfg.head_dim;
+  at.err = b.err;
+  if (route) {
+    at.route_ranks = route->ranks;
+    at.route_head0 = route->head0;
+    at.route_rows = route->rows;
+    at.route_ld = route->ld;
+    for (int r = 0; r < route->ranks; ++r) at.route_dst[r] = static_cast<__nv_bfloat16*>(route->dst[r]);
+  }
+  H3_TRY(mark(h, timing, 3, s));
   H3_TRY(h3::launch_attention(at, enc, s));
-  H3_TRY(mark(4));
+  H3_TRY(mark(h, timing, 4, s));
+  return H3BLK_OK;
+}
+
+int phase_out(const h3blk_ctx* h, const Span& sp, const void* x, const int32_t* tag, const int32_t* tidx,
+              const float* mod_table, const h3blk_weights* w, const BlockBufs& b, void* out, int sms,
+              PFN_cuTensorMapEncodeTiled_v12000 enc, cudaStream_t s, bool timing) {
+  const h3blk_config& c = h->cfg;
+  const bool q = c.quant != 0;
+  const size_t C = c.hidden, HD = (size_t)c.heads * c.head_dim, F = c.ffn;
+  const int64_t n = sp.n_local;
+  auto* xb = static_cast<const __nv_bfloat16*>(x);
+  const int32_t* tg = tag + sp.row0;
+  const int32_t* ti = tidx + sp.row0;
 
   // ---- out-projection + gated residual
-  if (q)
-    H3_TRY(h3::launch_rotate_quant(o, n_rows, (int)HD, reinterpret_cast<int8_t*>(buf(H3BLK_STAGE_O_Q8)),
-                                   reinterpret_cast<float*>(buf(H3BLK_STAGE_O_SCALE)), s));
-  g = base_gemm(h, err);
-  g.A = q ? (const void*)buf(H3BLK_STAGE_O_Q8) : (const void*)o;
+  if (q) H3_TRY(h3::launch_rotate_quant(b.o, n, (int)HD, b.o_q, b.o_s, s));
+  GemmArgs g = base_gemm(h, b.err);
+  g.A = q ? (const void*)b.o_q : (const void*)b.o;
   g.B = w->wo;
-  g.M = n_rows;
+  g.M = n;
   g.N = c.hidden;
   g.Nb = c.hidden;
   g.K = (int)HD;
   g.epi = h3::kEpiResid;
-  g.out = x1;
+  g.out = b.x1;
   g.ld_out = C;
   g.resid = xb;
   g.table = mod_table;
-  g.tag = tag;
-  g.tidx = tidx;
+  g.tag = tg;
+  g.tidx = ti;
   g.gate_idx = 2;
-  g.s_a = q ? reinterpret_cast<const float*>(buf(H3BLK_STAGE_O_SCALE)) : nullptr;
+  g.s_a = q ? b.o_s : nullptr;
   g.s_b = w->s_o;
-  H3_TRY(mark(5));
+  H3_TRY(mark(h, timing, 5, s));
   H3_TRY(h3::launch_gemm(g, enc, sms, s));
-  H3_TRY(mark(6));
+  H3_TRY(mark(h, timing, 6, s));
 
   // ---- pre-FFN AdaLN + RMSNorm
-  mn.x = x1;
+  h3::ModNormArgs mn;
+  std::memset(&mn, 0, sizeof(mn));
+  mn.x = b.x1;
+  mn.tag = tg;
+  mn.tidx = ti;
+  mn.table = mod_table;
+  mn.n = n;
+  mn.C = c.hidden;
+  mn.n_tags = c.n_tags;
+  mn.n_t = c.n_t;
   mn.shift_idx = 3;
   mn.scale_idx = 4;
-  if (q) {
-    mn.out_q = reinterpret_cast<int8_t*>(buf(H3BLK_STAGE_H2_Q8));
-    mn.out_scale = reinterpret_cast<float*>(buf(H3BLK_STAGE_H2_SCALE));
-  } else {
-    mn.out_bf16 = reinterpret_cast<__nv_bfloat16*>(buf(H3BLK_STAGE_H2));
-  }
+  mn.eps = c.norm_eps;
+  mn.out_q = b.h2_q;
+  mn.out_scale = b.h2_s;
+  mn.out_bf16 = q ? nullptr : b.h2;
   H3_TRY(h3::launch_modnorm(mn, s));
 
   // ---- FFN up (W1 | W3) + SwiGLU
-  g = base_gemm(h, err);
-  g.A = q ? (const void*)buf(H3BLK_STAGE_H2_Q8) : (const void*)buf(H3BLK_STAGE_H2);
+  g = base_gemm(h, b.err);
+  g.A = q ? (const void*)b.h2_q : (const void*)b.h2;
   g.B = w->w13;
-  g.M = n_rows;
+  g.M = n;
   g.N = c.ffn;
   g.Nb = 2 * c.ffn;
   g.K = c.hidden;
   g.epi = h3::kEpiSwiGLU;
-  g.out = a;
+  g.out = b.a;
   g.ld_out = F;
-  g.s_a = q ? reinterpret_cast<const float*>(buf(H3BLK_STAGE_H2_SCALE)) : nullptr;
+  g.s_a = q ? b.h2_s : nullptr;
   g.s_b = w->s_13;
-  H3_TRY(mark(7));
+  H3_TRY(mark(h, timing, 7, s));
   H3_TRY(h3::launch_gemm(g, enc, sms, s));
-  H3_TRY(mark(8));
+  H3_TRY(mark(h, timing, 8, s));
 
   // ---- FFN down + gated residual
-  if (q)
-    H3_TRY(h3::launch_rotate_quant(a, n_rows, (int)F, reinterpret_cast<int8_t*>(buf(H3BLK_STAGE_A_Q8)),
-                                   reinterpret_cast<float*>(buf(H3BLK_STAGE_A_SCALE)), s));
-  g = base_gemm(h, err);
-  g.A = q ? (const void*)buf(H3BLK_STAGE_A_Q8) : (const void*)a;
+  if (q) H3_TRY(h3::launch_rotate_quant(b.a, n, (int)F, b.a_q, b.a_s, s));
+  g = base_gemm(h, b.err);
+  g.A = q ? (const void*)b.a_q : (const void*)b.a;
   g.B = w->w2;
-  g.M = n_rows;
+  g.M = n;
   g.N = c.hidden;
   g.Nb = c.hidden;
   g.K = c.ffn;
   g.epi = h3::kEpiResid;
   g.out = out;
   g.ld_out = C;
-  g.resid = x1;
+  g.resid = b.x1;
   g.table = mod_table;
-  g.tag = tag;
-  g.tidx = tidx;
+  g.tag = tg;
+  g.tidx = ti;
   g.gate_idx = 5;
-  g.s_a = q ? reinterpret_cast<const float*>(buf(H3BLK_STAGE_A_SCALE)) : nullptr;
+  g.s_a = q ? b.a_s : nullptr;
   g.s_b = w->s_2;
-  H3_TRY(mark(9));
+  H3_TRY(mark(h, timing, 9, s));
   H3_TRY(h3::launch_gemm(g, enc, sms, s));
-  H3_TRY(mark(10));
+  H3_TRY(mark(h, timing, 10, s));
   return H3BLK_OK;
+}
+
+int block_forward(const h3blk_ctx* h, int64_t n_rows, const void* x, const int32_t* tag, const int32_t* tidx,
+                  const int32_t* pos, const float* mod_table, const h3blk_weights* w, void* out, void* workspace,
+                  int sms, PFN_cuTensorMapEncodeTiled_v12000 enc, cudaStream_t s, bool clear_err, bool timing) {
+  const Layout L = make_layout(h->cfg, n_rows);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  auto buf = [&](int stage) { return L.len[stage] ? ws + L.off[stage] : nullptr; };
+  BlockBufs b;
+  b.err = reinterpret_cast<int*>(buf(H3BLK_STAGE_ERROR));
+  b.tiles = reinterpret_cast<h3::TileInfo*>(ws + L.tiles_off);
+  b.h1 = reinterpret_cast<__nv_bfloat16*>(buf(H3BLK_STAGE_H1));
+  b.qkv = reinterpret_cast<__nv_bfloat16*>(buf(H3BLK_STAGE_QKV));
+  b.o = reinterpret_cast<__nv_bfloat16*>(buf(H3BLK_STAGE_O));
+  b.x1 = reinterpret_cast<__nv_bfloat16*>(buf(H3BLK_STAGE_X1));
+  b.h2 = reinterpret_cast<__nv_bfloat16*>(buf(H3BLK_STAGE_H2));
+  b.a = reinterpret_cast<__nv_bfloat16*>(buf(H3BLK_STAGE_A));
+  b.h1_q = reinterpret_cast<int8_t*>(buf(H3BLK_STAGE_H1_Q8));
+  b.o_q = reinterpret_cast<int8_t*>(buf(H3BLK_STAGE_O_Q8));
+  b.h2_q = reinterpret_cast<int8_t*>(buf(H3BLK_STAGE_H2_Q8));
+  b.a_q = reinterpret_cast<int8_t*>(buf(H3BLK_STAGE_A_Q8));
+  b.h1_s = reinterpret_cast<float*>(buf(H3BLK_STAGE_H1_SCALE));
+  b.o_s = reinterpret_cast<float*>(buf(H3BLK_STAGE_O_SCALE));
+  b.h2_s = reinterpret_cast<float*>(buf(H3BLK_STAGE_H2_SCALE));
+  b.a_s = reinterpret_cast<float*>(buf(H3BLK_STAGE_A_SCALE));
+  const Span sp{n_rows, 0, n_rows};
+  int st = phase_qkv(h, sp, x, tag, tidx, pos, mod_table, w, b, nullptr, sms, enc, s, clear_err, timing);
+  if (st != H3BLK_OK) return st;
+  st = phase_attention(h, n_rows, h->cfg.heads, tag, b, nullptr, enc, s, timing);
+  if (st != H3BLK_OK) return st;
+  return phase_out(h, sp, x, tag, tidx, mod_table, w, b, out, sms, enc, s, timing);
 }
 
 }  // namespace h3api

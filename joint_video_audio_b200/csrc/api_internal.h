@@ -29,6 +29,50 @@ int check_block_weights(const h3blk_config& c, const h3blk_weights* w);
 // Bytes of one block forward's workspace over n rows (error word at offset 0).
 size_t block_workspace_bytes(const h3blk_config& c, int64_t n);
 
+// Buffers of one block forward (W8A8 ones null in bf16 mode and vice versa).
+struct BlockBufs {
+  int* err;
+  h3::TileInfo* tiles;
+  __nv_bfloat16 *h1, *qkv, *o, *x1, *h2, *a;
+  int8_t *h1_q, *o_q, *h2_q, *a_q;
+  float *h1_s, *o_s, *h2_s, *a_s;
+};
+
+// This call's rows [row0, row0 + n_local) of a packed sequence of n_total rows.
+struct Span {
+  int64_t n_local, row0, n_total;
+};
+
+// Head-group routing of the QKV projection: head h goes to dst[h / hg], a
+// [n_total, 3 * hg * head_dim] buffer, at its global row.
+struct QkvRoute {
+  int ranks, hg;
+  void* dst[h3::kMaxRanks];
+};
+
+// Row routing of the attention output: global row r goes to
+// dst[r / rows] at row r % rows of a [rows, ld] buffer, columns from
+// (head0 + head) * head_dim.
+struct ORoute {
+  int ranks, head0;
+  int64_t rows, ld;
+  void* dst[h3::kMaxRanks];
+};
+
+// The block in three phases: tile summary + pre-norm + QKV (x = this call's
+// rows; tag / tidx / pos cover the whole sequence), attention over the whole
+// sequence for `heads` heads, and out-projection through the FFN for this
+// call's rows.
+int phase_qkv(const h3blk_ctx* h, const Span& sp, const void* x, const int32_t* tag, const int32_t* tidx,
+              const int32_t* pos, const float* mod_table, const h3blk_weights* w, const BlockBufs& b,
+              const QkvRoute* route, int sms, PFN_cuTensorMapEncodeTiled_v12000 enc, cudaStream_t s, bool clear_err,
+              bool timing);
+int phase_attention(const h3blk_ctx* h, int64_t n_total, int heads, const int32_t* tag, const BlockBufs& b,
+                    const ORoute* route, PFN_cuTensorMapEncodeTiled_v12000 enc, cudaStream_t s, bool timing);
+int phase_out(const h3blk_ctx* h, const Span& sp, const void* x, const int32_t* tag, const int32_t* tidx,
+              const float* mod_table, const h3blk_weights* w, const BlockBufs& b, void* out, int sms,
+              PFN_cuTensorMapEncodeTiled_v12000 enc, cudaStream_t s, bool timing);
+
 // The block forward's launch sequence on validated arguments. clear_err resets
 // the error word (offset 0 of the workspace) first; timing records the
 // handle's events.

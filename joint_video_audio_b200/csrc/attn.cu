@@ -382,7 +382,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     } else if (mbar_wait(s.o_final, 0, abort)) {
       tc_fence_after();
       const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
-      __nv_bfloat16* dst = p.o + row * (int64_t)HD + head * D;
+      __nv_bfloat16* dst;
+      if (p.route_ranks > 0) {
+        // sequence parallelism: the row's owner gathers every head group's output
+        const int64_t d = row / p.route_rows;
+        dst = p.route_dst[row_ok ? d : 0] + (row - d * p.route_rows) * p.route_ld + (int64_t)(p.route_head0 + head) * D;
+      } else {
+        dst = p.o + row * (int64_t)HD + head * D;
+      }
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];

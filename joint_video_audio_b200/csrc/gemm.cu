@@ -15,7 +15,10 @@
 // page, constructor: qk_norm_eps of the per-head query/key norms, rope_theta;
 // introduction: AdaLN modulation per modality tag; ffn_dim of the SwiGLU):
 //   kEpiQKV    q, k: per-head RMSNorm (fp32) * gain, then 3D RoPE on adjacent
-//              pairs; v: stored as is. Output [M, 3*H*D] bf16.
+//              pairs; v: stored as is. Output [M, 3*H*D] bf16, or, routed by
+//              head group for sequence parallelism, each head's q / k / v to
+//              its group owner's [rows, 3*Hg*D] buffer (peer memory or a send
+//              buffer).
 //   kEpiResid  out = resid + gate[tag][tidx] * acc (padding rows: out = resid).
 //   kEpiSwiGLU B holds W1 rows then W3 rows; tile j loads W1 rows j*128.. and W3
 //              rows j*128.. into its two 128-column halves: out = silu(g) * u.
@@ -218,7 +221,17 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tacc, 
       if (col0 >= p.N) break;
       const int region = col0 / p.hd;  // 0 q, 1 k, 2 v
       const uint32_t th = tacc + hh * D;
-      __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + row * p.ld_out + col0;
+      __nv_bfloat16* dst;
+      if (p.route_ranks > 0) {
+        // sequence parallelism: the head's group owner holds q / k / v of
+        // every row for its heads
+        const int hi = (col0 - region * p.hd) / D;
+        const int hg = p.route_hg;
+        dst = reinterpret_cast<__nv_bfloat16*>(p.route_dst[hi / hg]) +
+              (p.route_row0 + row) * (int64_t)(3 * hg * D) + (region * hg + hi % hg) * D;
+      } else {
+        dst = reinterpret_cast<__nv_bfloat16*>(p.out) + row * p.ld_out + col0;
+      }
       if (region == 2) {
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {

@@ -9,6 +9,7 @@
 namespace h3 {
 
 constexpr int kMaxRopePairs = 128;  // head_dim <= 256
+constexpr int kMaxRanks = 8;        // ranks of a sequence-parallel (Ulysses) group
 
 // Rotary table of one head: for pair j, which position axis drives it
 // (0 t, 1 h, 2 w, 3 none) and its frequency.
@@ -96,6 +97,12 @@ struct GemmArgs {
   const float* s_a;
   const float* s_b;
   int* err;
+  // kEpiQKV routing by head group (route_ranks > 0): head h of region q / k / v
+  // goes to route_dst[h / route_hg], a [rows, 3 * route_hg * head_dim] buffer,
+  // at row route_row0 + row
+  int route_ranks = 0, route_hg = 0;
+  int64_t route_row0 = 0;
+  void* route_dst[kMaxRanks] = {};
 };
 cudaError_t launch_gemm(const GemmArgs& a, PFN_cuTensorMapEncodeTiled_v12000 encode, int num_sms, cudaStream_t s);
 
@@ -108,6 +115,12 @@ struct AttnArgs {
   int64_t n;
   int heads, head_dim;
   int* err;
+  // output routing by row (route_ranks > 0): row r goes to
+  // route_dst[r / route_rows] at row r % route_rows of a [route_rows, route_ld]
+  // buffer, columns from (route_head0 + head) * head_dim
+  int route_ranks = 0, route_head0 = 0;
+  int64_t route_rows = 0, route_ld = 0;
+  __nv_bfloat16* route_dst[kMaxRanks] = {};
 };
 cudaError_t launch_attention(const AttnArgs& a, PFN_cuTensorMapEncodeTiled_v12000 encode, cudaStream_t s);
 

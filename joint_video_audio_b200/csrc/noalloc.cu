@@ -96,7 +96,7 @@ extern "C" int h3blk_attention_noalloc(int64_t n_rows, int heads, int head_dim, 
   // the error word must start at zero; the tile summary is rewritten in full
   if (cudaMemsetAsync(err, 0, sizeof(int), s) != cudaSuccess) return H3BLK_ERR_CUDA;
   if (h3::launch_tile_info(tag, tidx, n_rows, n_tags, n_t, tiles, err, s) != cudaSuccess) return H3BLK_ERR_CUDA;
-  h3::AttnArgs a;
+  h3::AttnArgs a{};  // every field not set below (output routing among them) stays zero
   a.qkv = static_cast<const __nv_bfloat16*>(qkv);
   a.o = static_cast<__nv_bfloat16*>(o);
   a.tag = tag;

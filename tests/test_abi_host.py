@@ -286,3 +286,63 @@ def test_model_graph_create_validates_before_capture():
     assert e.value.status == B.H3BLK_ERR_INVALID_ARG
     assert B.h3blk_graph_launch(None, None) == B.H3BLK_ERR_INVALID_ARG
     B.h3blk_graph_destroy(None)   # no-op
+
+
+# ---------------------------------------------------------------- sequence parallelism
+
+def test_ulysses_sizes_and_group_checks():
+    blk = j.H3Block(hi.TINY)   # 6 heads of 64
+    q, o = B.h3blk_ulysses_buffer_bytes(blk.handle, 320, 2)
+    assert q == 320 * 3 * 3 * 64 * 2 and o == 160 * 6 * 64 * 2
+    assert B.h3blk_ulysses_workspace_bytes(blk.handle, 320, 2) < blk.workspace_bytes(320)
+    for n, world in ((320, 4), (322, 3)):
+        with pytest.raises(B.H3BlkError) as e:
+            B.h3blk_ulysses_buffer_bytes(blk.handle, n, world)
+        assert e.value.status == B.H3BLK_ERR_UNSUPPORTED
+    with pytest.raises(B.H3BlkError):
+        B.h3blk_ulysses_workspace_bytes(blk.handle, 320, 9)
+
+
+def _fake_ulysses(world=2, rank=0):
+    base = 1 << 40
+    p = lambda k: base + (k << 28)  # noqa: E731
+    u = B.h3blk_ulysses(world=world, rank=rank)
+    for d in range(world):
+        u.qkv[d] = p(40 + d)
+        u.o[d] = p(50 + d)
+    w = B.h3blk_weights(wqkv=p(1), q_gain=p(2), k_gain=p(3), wo=p(4), w13=p(5), w2=p(6))
+    return u, w, p
+
+
+@pytest.mark.parametrize("case,status", [
+    ("ok", B.H3BLK_ERR_CUDA),                     # passes every host check, fails at the first CUDA call
+    ("rank_out_of_group", B.H3BLK_ERR_INVALID_ARG),
+    ("missing_peer_qkv", B.H3BLK_ERR_INVALID_ARG),
+    ("misaligned_peer", B.H3BLK_ERR_INVALID_ARG),
+    ("workspace_too_small", B.H3BLK_ERR_INVALID_ARG),
+    ("world_not_dividing_heads", B.H3BLK_ERR_UNSUPPORTED),
+])
+def test_ulysses_phases_validate_before_gpu(case, status):
+    blk = j.H3Block(hi.TINY)
+    u, w, p = _fake_ulysses()
+    ws = B.h3blk_ulysses_workspace_bytes(blk.handle, 320, 2)
+    if case == "rank_out_of_group":
+        u.rank = 2
+    if case == "missing_peer_qkv":
+        u.qkv[1] = None
+    if case == "misaligned_peer":
+        u.qkv[1] = p(41) + 8
+        u.o[1] = p(51) + 8
+    if case == "workspace_too_small":
+        ws = 64
+    if case == "world_not_dividing_heads":
+        u.world = 4
+        u.qkv[2], u.qkv[3], u.o[2], u.o[3] = p(42), p(43), p(52), p(53)
+    st = B.h3blk_ulysses_qkv(blk.handle, 320, u, p(10), p(11), p(12), p(13), p(14), w, p(20), ws, None)
+    assert st == status
+    if case in ("ok", "rank_out_of_group", "misaligned_peer", "workspace_too_small", "world_not_dividing_heads"):
+        assert B.h3blk_ulysses_attention(blk.handle, 320, u, p(11), p(20), ws, None) == status
+        # the output phase reads only this rank's own o buffer
+        st_out = B.H3BLK_ERR_CUDA if case == "misaligned_peer" else status
+        assert B.h3blk_ulysses_out(blk.handle, 320, u, p(10), p(11), p(12), p(14), w, p(15), p(20), ws,
+                                   None) == st_out
