@@ -13,3 +13,4 @@ from .h3_modulation import (  # noqa: F401
     modulation_table, produce, sinusoidal_embedding, time_mlp, timestep_frequencies, two_time_embedding,
 )
 from .h3_model import ModelOracle, affine, norm_out, refine_text, scatter_rows  # noqa: F401
+from .h3_sparse import block_scores, select, sparse_attention, sparse_block_attention  # noqa: F401
