@@ -132,7 +132,10 @@ H3BLK_API int h3blk_workspace_bytes(h3blk_handle h, int64_t n_rows, size_t* byte
  *   H3BLK_STAGE_A              bf16 [N, F]      SwiGLU output
  *   H3BLK_STAGE_*_Q8           int8 [N, K]      rotated, quantised linear input (W8A8)
  *   H3BLK_STAGE_*_SCALE        fp32 [N]         its per-row scale            (W8A8)
- *   H3BLK_STAGE_ERROR          int32 [1]        device error bits of the last forward */
+ *   H3BLK_STAGE_ERROR          int32 [1]        device error bits of the last forward
+ *   H3BLK_STAGE_KV_LIST        int32 [ceil(N/256)][H][1 + ceil(N/128)]  block-sparse mode
+ *                              only: per 256-query block and head, the count of
+ *                              kept 128-key tiles, then the tiles ascending */
 enum {
   H3BLK_STAGE_H1 = 0,
   H3BLK_STAGE_QKV = 1,
@@ -149,7 +152,8 @@ enum {
   H3BLK_STAGE_A_Q8 = 12,
   H3BLK_STAGE_A_SCALE = 13,
   H3BLK_STAGE_ERROR = 14,
-  H3BLK_STAGE_COUNT = 15
+  H3BLK_STAGE_KV_LIST = 15,
+  H3BLK_STAGE_COUNT = 16
 };
 H3BLK_API int h3blk_stage_view(h3blk_handle h, int64_t n_rows, int stage, size_t* offset, size_t* bytes);
 
@@ -173,6 +177,20 @@ H3BLK_API int h3blk_forward(h3blk_handle h, int64_t n_rows, const void* x, const
  * that used `workspace`: *status = H3BLK_OK, H3BLK_ERR_BAD_INDEX or
  * H3BLK_ERR_TIMEOUT. */
 H3BLK_API int h3blk_check(h3blk_handle h, int64_t n_rows, const void* workspace, void* stream, int* status);
+
+/* Block-sparse attention for later forwards on this handle (the optional
+ * sparse backend of "HyperFlow for MiniMax-H3", model card: summary table and
+ * Performance; its method is not described there, so this is this library's
+ * reading). density = 1 (the default) is dense attention. For 0 < density < 1,
+ * every 256-query block keeps, per head, k = max(1, ceil(n * m / 1024)) of the
+ * n 128-key tiles that hold a valid row, m = round(1024 * density): those
+ * whose mean key has the largest dot product with the block's mean query
+ * (means over valid rows; ties toward the lower tile). Valid rows then attend
+ * only to the valid keys of the kept tiles; padding rows' attention output is
+ * undefined (the block's zero gates discard it). The workspace grows
+ * (h3blk_workspace_bytes follows the setting). INVALID_ARG unless
+ * 0 < density <= 1; UNSUPPORTED for the sequence-parallel calls. */
+H3BLK_API int h3blk_set_attention_density(h3blk_handle h, float density);
 
 /* Per-kernel timing. When set, every later h3blk_forward on this handle
  * records the caller's CUDA events (cudaEvent_t passed as void*) on its stream

@@ -20,7 +20,7 @@ H3BLK_ERR_TIMEOUT = 4
 H3BLK_ERR_BAD_INDEX = 5
 
 STAGES = ["H1", "QKV", "O", "X1", "H2", "A", "H1_Q8", "H1_SCALE", "O_Q8", "O_SCALE",
-          "H2_Q8", "H2_SCALE", "A_Q8", "A_SCALE", "ERROR"]
+          "H2_Q8", "H2_SCALE", "A_Q8", "A_SCALE", "ERROR", "KV_LIST"]
 STAGE = {name: i for i, name in enumerate(STAGES)}
 
 # every symbol include/h3blk.h declares
@@ -31,7 +31,7 @@ EXPORTS = ["h3blk_create", "h3blk_destroy", "h3blk_workspace_bytes", "h3blk_stag
            "h3blk_modulation_table", "h3blk_model_workspace_bytes", "h3blk_model_forward", "h3blk_model_check",
            "h3blk_model_graph_create", "h3blk_graph_launch", "h3blk_graph_info", "h3blk_graph_destroy",
            "h3blk_ulysses_buffer_bytes", "h3blk_ulysses_workspace_bytes", "h3blk_ulysses_qkv",
-           "h3blk_ulysses_attention", "h3blk_ulysses_out"]
+           "h3blk_ulysses_attention", "h3blk_ulysses_out", "h3blk_set_attention_density"]
 
 H3BLK_MAX_RANKS = 8
 
@@ -132,6 +132,7 @@ def _load():
         "h3blk_graph_launch": (i32, [vp, vp]),
         "h3blk_graph_info": (i32, [vp, C.POINTER(i32), C.POINTER(i32)]),
         "h3blk_graph_destroy": (None, [vp]),
+        "h3blk_set_attention_density": (i32, [vp, C.c_float]),
         "h3blk_ulysses_buffer_bytes": (i32, [vp, i64, i32, C.POINTER(sz), C.POINTER(sz)]),
         "h3blk_ulysses_workspace_bytes": (i32, [vp, i64, i32, C.POINTER(sz)]),
         "h3blk_ulysses_qkv": (i32, [vp, i64, C.POINTER(h3blk_ulysses), vp, vp, vp, vp, vp, C.POINTER(h3blk_weights),
@@ -335,3 +336,7 @@ def h3blk_ulysses_out(handle, n_rows, u, x_local, tag, tidx, table, w, out_local
                       stream) -> int:
     return _lib.h3blk_ulysses_out(handle, n_rows, C.byref(u), x_local, tag, tidx, table, C.byref(w), out_local,
                                   workspace, workspace_bytes, stream)
+
+
+def h3blk_set_attention_density(handle, density) -> int:
+    return _lib.h3blk_set_attention_density(handle, C.c_float(density))

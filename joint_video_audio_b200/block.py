@@ -59,6 +59,14 @@ class H3Block:
             B.h3blk_destroy(h)
             self.handle = None
 
+    # ------------------------------------------------------------ attention mode
+    def set_attention_density(self, density: float) -> None:
+        """1.0: dense attention; below: block-sparse (h3blk_set_attention_density).
+        The workspace size follows the setting."""
+        st = B.h3blk_set_attention_density(self.handle, float(density))
+        if st != B.H3BLK_OK:
+            raise B.H3BlkError("h3blk_set_attention_density", st)
+
     # ------------------------------------------------------------ workspace
     def workspace_bytes(self, n_rows: int) -> int:
         return B.h3blk_workspace_bytes(self.handle, n_rows)
@@ -76,11 +84,14 @@ class H3Block:
                   "QKV": ("bf16", 3 * hd), "O": ("bf16", hd), "A": ("bf16", d.ffn),
                   "H1_Q8": ("i8", d.hidden), "H2_Q8": ("i8", d.hidden), "O_Q8": ("i8", hd), "A_Q8": ("i8", d.ffn),
                   "H1_SCALE": ("f32", 1), "H2_SCALE": ("f32", 1), "O_SCALE": ("f32", 1), "A_SCALE": ("f32", 1),
-                  "ERROR": ("i32", 1)}
+                  "ERROR": ("i32", 1), "KV_LIST": ("i32", 1)}
         dt, cols = shapes[name]
         v = raw.view(_DT[dt])
         if name == "ERROR":
             return v
+        if name == "KV_LIST":
+            n_tiles = (n_rows + 127) // 128
+            return v.view((n_tiles + 1) // 2, d.heads, 1 + n_tiles)
         return v.view(n_rows, cols) if cols > 1 else v.view(n_rows)
 
     # ------------------------------------------------------------ int8 weights

@@ -82,10 +82,11 @@ struct Layout {
   size_t off[H3BLK_STAGE_COUNT];
   size_t len[H3BLK_STAGE_COUNT];
   size_t tiles_off;
+  size_t sp_qsum, sp_ksum, sp_count;  // block-sparse pooling buffers (0 when dense)
   size_t total;
 };
 
-Layout make_layout(const h3blk_config& c, int64_t n) {
+Layout make_layout(const h3blk_config& c, int64_t n, int keep_per_1024) {
   Layout L;
   std::memset(&L, 0, sizeof(L));
   const size_t N = (size_t)n, C = c.hidden, HD = (size_t)c.heads * c.head_dim, F = c.ffn;
@@ -114,6 +115,17 @@ Layout make_layout(const h3blk_config& c, int64_t n) {
     put(H3BLK_STAGE_H2_SCALE, N * 4);
     put(H3BLK_STAGE_A_Q8, N * F);
     put(H3BLK_STAGE_A_SCALE, N * 4);
+  }
+  if (keep_per_1024 < 1024) {
+    const size_t n_tiles = (N + 127) / 128, n_blocks = (n_tiles + 1) / 2, H = c.heads;
+    const size_t pool = n_tiles * H * (size_t)c.head_dim * 4;
+    L.sp_qsum = o;
+    o = align256(o + pool);
+    L.sp_ksum = o;
+    o = align256(o + pool);
+    L.sp_count = o;
+    o = align256(o + n_tiles * 4);
+    put(H3BLK_STAGE_KV_LIST, n_blocks * H * (1 + n_tiles) * 4);
   }
   L.total = o;
   return L;
@@ -174,7 +186,9 @@ int check_block_weights(const h3blk_config& c, const h3blk_weights* w) {
   return H3BLK_OK;
 }
 
-size_t block_workspace_bytes(const h3blk_config& c, int64_t n) { return make_layout(c, n).total; }
+size_t block_workspace_bytes(const h3blk_config& c, int64_t n, int keep_per_1024) {
+  return make_layout(c, n, keep_per_1024).total;
+}
 
 #define H3_TRY(expr)                              \
   do {                                            \
@@ -268,6 +282,25 @@ int phase_attention(const h3blk_ctx* h, int64_t n_total, int heads, const int32_
     for (int r = 0; r < route->ranks; ++r) at.route_dst[r] = static_cast<__nv_bfloat16*>(route->dst[r]);
   }
   H3_TRY(mark(h, timing, 3, s));
+  if (b.sp_lists) {
+    // block-sparse: pool q and k per tile, rank the tiles per block and head
+    h3::SparseArgs sa;
+    std::memset(&sa, 0, sizeof(sa));
+    sa.qkv = b.qkv;
+    sa.tag = tag;
+    sa.n = n_total;
+    sa.heads = heads;
+    sa.head_dim = h->cfg.head_dim;
+    sa.keep_per_1024 = h->keep_per_1024;
+    sa.qsum = b.sp_qsum;
+    sa.ksum = b.sp_ksum;
+    sa.count = b.sp_count;
+    sa.lists = b.sp_lists;
+    sa.list_stride = 1 + (n_total + 127) / 128;
+    H3_TRY(h3::launch_sparse_select(sa, s));
+    at.kv_list = b.sp_lists;
+    at.kv_list_stride = sa.list_stride;
+  }
   H3_TRY(h3::launch_attention(at, enc, s));
   H3_TRY(mark(h, timing, 4, s));
   return H3BLK_OK;
@@ -371,12 +404,17 @@ int phase_out(const h3blk_ctx* h, const Span& sp, const void* x, const int32_t* 
 int block_forward(const h3blk_ctx* h, int64_t n_rows, const void* x, const int32_t* tag, const int32_t* tidx,
                   const int32_t* pos, const float* mod_table, const h3blk_weights* w, void* out, void* workspace,
                   int sms, PFN_cuTensorMapEncodeTiled_v12000 enc, cudaStream_t s, bool clear_err, bool timing) {
-  const Layout L = make_layout(h->cfg, n_rows);
+  const Layout L = make_layout(h->cfg, n_rows, h->keep_per_1024);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   auto buf = [&](int stage) { return L.len[stage] ? ws + L.off[stage] : nullptr; };
-  BlockBufs b;
+  BlockBufs b{};
   b.err = reinterpret_cast<int*>(buf(H3BLK_STAGE_ERROR));
   b.tiles = reinterpret_cast<h3::TileInfo*>(ws + L.tiles_off);
+  const bool sparse = h->keep_per_1024 < 1024;
+  b.sp_qsum = sparse ? reinterpret_cast<float*>(ws + L.sp_qsum) : nullptr;
+  b.sp_ksum = sparse ? reinterpret_cast<float*>(ws + L.sp_ksum) : nullptr;
+  b.sp_count = sparse ? reinterpret_cast<int32_t*>(ws + L.sp_count) : nullptr;
+  b.sp_lists = reinterpret_cast<int32_t*>(buf(H3BLK_STAGE_KV_LIST));
   b.h1 = reinterpret_cast<__nv_bfloat16*>(buf(H3BLK_STAGE_H1));
   b.qkv = reinterpret_cast<__nv_bfloat16*>(buf(H3BLK_STAGE_QKV));
   b.o = reinterpret_cast<__nv_bfloat16*>(buf(H3BLK_STAGE_O));
@@ -443,6 +481,7 @@ int h3blk_create(const h3blk_config* cfg, h3blk_handle* out) {
   if (!h) return H3BLK_ERR_INVALID_ARG;
   h->cfg = c;
   h->timing = false;
+  h->keep_per_1024 = 1024;
   for (auto& e : h->events) e = nullptr;
   const int pairs[3] = {c.rope_pairs_t, c.rope_pairs_h, c.rope_pairs_w};
   int j = 0;
@@ -476,15 +515,24 @@ int h3blk_set_kernel_events(h3blk_handle h, void* const* events, int n_events) {
   return H3BLK_OK;
 }
 
+int h3blk_set_attention_density(h3blk_handle h, float density) {
+  if (!h || !(density > 0.f && density <= 1.f)) return H3BLK_ERR_INVALID_ARG;
+  int m = (int)std::lround((double)density * 1024.0);
+  if (m < 1) m = 1;
+  if (m > 1024) m = 1024;
+  h->keep_per_1024 = m;
+  return H3BLK_OK;
+}
+
 int h3blk_workspace_bytes(h3blk_handle h, int64_t n_rows, size_t* bytes) {
   if (!h || !bytes || n_rows < 1) return H3BLK_ERR_INVALID_ARG;
-  *bytes = make_layout(h->cfg, n_rows).total;
+  *bytes = make_layout(h->cfg, n_rows, h->keep_per_1024).total;
   return H3BLK_OK;
 }
 
 int h3blk_stage_view(h3blk_handle h, int64_t n_rows, int stage, size_t* offset, size_t* bytes) {
   if (!h || !offset || !bytes || n_rows < 1 || stage < 0 || stage >= H3BLK_STAGE_COUNT) return H3BLK_ERR_INVALID_ARG;
-  const Layout L = make_layout(h->cfg, n_rows);
+  const Layout L = make_layout(h->cfg, n_rows, h->keep_per_1024);
   if (L.len[stage] == 0) return H3BLK_ERR_UNSUPPORTED;  // stage not produced in this mode
   *offset = L.off[stage];
   *bytes = L.len[stage];
@@ -501,7 +549,7 @@ int h3blk_forward(h3blk_handle h, int64_t n_rows, const void* x, const int32_t* 
   const void* ptrs[] = {x, tag, tidx, pos, mod_table, out, workspace};
   for (const void* p : ptrs)
     if (!aligned16(p)) return H3BLK_ERR_INVALID_ARG;
-  const Layout L = make_layout(c, n_rows);
+  const Layout L = make_layout(c, n_rows, h->keep_per_1024);
   if (workspace_bytes < L.total) return H3BLK_ERR_INVALID_ARG;
   const size_t N = (size_t)n_rows, C = c.hidden;
   if (overlap(out, N * C * 2, x, N * C * 2) || overlap(out, N * C * 2, workspace, L.total) ||
@@ -518,7 +566,7 @@ int h3blk_forward(h3blk_handle h, int64_t n_rows, const void* x, const int32_t* 
 
 int h3blk_check(h3blk_handle h, int64_t n_rows, const void* workspace, void* stream, int* status) {
   if (!h || !workspace || !status || n_rows < 1) return H3BLK_ERR_INVALID_ARG;
-  const Layout L = make_layout(h->cfg, n_rows);
+  const Layout L = make_layout(h->cfg, n_rows, h->keep_per_1024);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(s) != cudaSuccess) return H3BLK_ERR_CUDA;
   int bits = 0;

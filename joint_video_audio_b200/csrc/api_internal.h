@@ -12,6 +12,7 @@ struct h3blk_ctx {
   h3::RopeTable rope;
   cudaEvent_t events[H3BLK_TIMING_POINTS];
   bool timing;
+  int keep_per_1024;  // 1024: dense attention; below: block-sparse
 };
 
 namespace h3api {
@@ -26,16 +27,20 @@ int cuda_status(cudaError_t e);
 // Non-null, 16-byte aligned block weights (and int8 scales in W8A8 mode).
 int check_block_weights(const h3blk_config& c, const h3blk_weights* w);
 
-// Bytes of one block forward's workspace over n rows (error word at offset 0).
-size_t block_workspace_bytes(const h3blk_config& c, int64_t n);
+// Bytes of one block forward's workspace over n rows (error word at offset 0);
+// keep_per_1024 < 1024 adds the block-sparse selection buffers.
+size_t block_workspace_bytes(const h3blk_config& c, int64_t n, int keep_per_1024);
 
 // Buffers of one block forward (W8A8 ones null in bf16 mode and vice versa).
 struct BlockBufs {
-  int* err;
-  h3::TileInfo* tiles;
-  __nv_bfloat16 *h1, *qkv, *o, *x1, *h2, *a;
-  int8_t *h1_q, *o_q, *h2_q, *a_q;
-  float *h1_s, *o_s, *h2_s, *a_s;
+  int* err = nullptr;
+  h3::TileInfo* tiles = nullptr;
+  // block-sparse selection (null when dense)
+  float *sp_qsum = nullptr, *sp_ksum = nullptr;
+  int32_t *sp_count = nullptr, *sp_lists = nullptr;
+  __nv_bfloat16 *h1 = nullptr, *qkv = nullptr, *o = nullptr, *x1 = nullptr, *h2 = nullptr, *a = nullptr;
+  int8_t *h1_q = nullptr, *o_q = nullptr, *h2_q = nullptr, *a_q = nullptr;
+  float *h1_s = nullptr, *o_s = nullptr, *h2_s = nullptr, *a_s = nullptr;
 };
 
 // This call's rows [row0, row0 + n_local) of a packed sequence of n_total rows.

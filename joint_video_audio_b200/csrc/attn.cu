@@ -35,7 +35,8 @@
 // KV tiles whose rows all lie in the other document are skipped when neither
 // query tile needs them; tiles that mix documents, run past the end of the
 // sequence, or belong to the other document of one of the two query tiles are
-// masked per element.
+// masked per element. In block-sparse mode the CTA visits only the tiles of its
+// list (chosen in sparse.cu), with the same per-element masks.
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 #include <math_constants.h>
@@ -111,6 +112,20 @@ __device__ __forceinline__ int count_kv_tiles(const TileInfo* tiles, int n_tiles
   return n;
 }
 
+// The KV tiles one CTA visits, in order: every tile one of its two query
+// tiles needs (dense), or the tiles its block keeps (block-sparse list).
+struct KvSeq {
+  const TileInfo* tiles;
+  int n_tiles, qk0, qk1;
+  const int32_t* list;  // [count, tile, tile, ...] or nullptr
+  __device__ int count() const { return list ? list[0] : count_kv_tiles(tiles, n_tiles, qk0, qk1); }
+  // the tile of step j, given the tile of step j - 1 (-1 before the first)
+  __device__ int at(int j, int prev) const {
+    if (list) return j < list[0] ? list[1 + j] : n_tiles;
+    return next_kv_tile(tiles, n_tiles, qk0, qk1, prev + 1);
+  }
+};
+
 __device__ __forceinline__ void fail(int* err, volatile int* abort) {
   if (err) atomicOr(err, kErrTimeoutAttn);
   *abort = 1;
@@ -156,7 +171,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *s.tmem_base;
-  const int n_kv = count_kv_tiles(p.tiles, n_tiles, qk0, qk1);
+  const KvSeq seq{p.tiles, n_tiles, qk0, qk1,
+                  p.kv_list ? p.kv_list + ((int64_t)pair * p.heads + head) * p.kv_list_stride : nullptr};
+  const int n_kv = seq.count();
 
   if (warp == 0) {
     // ------------------------------------------------------------ loads
@@ -170,8 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         for (int r = 0; r < kRegions; ++r)
           tma_load_2d(s.q0 + t * SM::kQBytes + r * SM::kRegion, &tm, s.q_full, head * D + r * 64, (qt0 + t) * kTile);
       int u = 0;
-      for (int kt = next_kv_tile(p.tiles, n_tiles, qk0, qk1, 0); kt < n_tiles;
-           kt = next_kv_tile(p.tiles, n_tiles, qk0, qk1, kt + 1)) {
+      for (int jj = 0, kt = seq.at(0, -1); kt < n_tiles; ++jj, kt = seq.at(jj, kt)) {
         bool ok = true;
         for (int kv = 0; kv < 2; ++kv, ++u) {  // K_j then V_j
           const int sl = u % kSlots;
@@ -279,14 +295,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     float m_run = -CUDART_INF_F, l_run = 0.f;
     bool ok = true;
     int j = 0;
-    int kt = next_kv_tile(p.tiles, n_tiles, qk0, qk1, 0);
+    int kt = seq.at(0, -1);
     TileInfo ti_next;
     if (kt < n_tiles) ti_next = p.tiles[kt];
     for (; kt < n_tiles; ++j) {
       const TileInfo ti = ti_next;
       // the next KV tile's summary is fetched before waiting for S, so its
       // global-memory latency hides behind the wait
-      const int kt_next = next_kv_tile(p.tiles, n_tiles, qk0, qk1, kt + 1);
+      const int kt_next = seq.at(j + 1, kt);
       if (kt_next < n_tiles) ti_next = p.tiles[kt_next];
       if (!mbar_wait(&s.s_full[t], j & 1, abort)) {
         ok = false;

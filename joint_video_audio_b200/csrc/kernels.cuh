@@ -121,8 +121,29 @@ struct AttnArgs {
   int route_ranks = 0, route_head0 = 0;
   int64_t route_rows = 0, route_ld = 0;
   __nv_bfloat16* route_dst[kMaxRanks] = {};
+  // block-sparse mode (kv_list != nullptr): the KV tiles of CTA (pair, head)
+  // are kv_list[(pair * heads + head) * kv_list_stride + 1 ..][0 .. count),
+  // count at offset 0, ascending
+  const int32_t* kv_list = nullptr;
+  int64_t kv_list_stride = 0;
 };
 cudaError_t launch_attention(const AttnArgs& a, PFN_cuTensorMapEncodeTiled_v12000 encode, cudaStream_t s);
+
+// ---------------------------------------------------------------- sparse selection
+// Per 256-query block and head, the 128-key tiles block-sparse attention keeps
+// (see sparse.cu): lists [n_blocks][heads][1 + n_tiles] as count, tiles.
+struct SparseArgs {
+  const __nv_bfloat16* qkv;  // [n, 3 * heads * head_dim], q and k final (normed, rotated)
+  const int32_t* tag;
+  int64_t n;
+  int heads, head_dim, keep_per_1024;
+  float* qsum;               // [n_tiles][heads][head_dim]
+  float* ksum;               // [n_tiles][heads][head_dim]
+  int32_t* count;            // [n_tiles] valid rows
+  int32_t* lists;
+  int64_t list_stride;       // 1 + n_tiles
+};
+cudaError_t launch_sparse_select(const SparseArgs& a, cudaStream_t s);
 
 // ---------------------------------------------------------------- modulation table
 constexpr int kMaxModSets = 8;  // timestep sets (the table's n_t) per call

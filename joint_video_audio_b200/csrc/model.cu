@@ -28,13 +28,13 @@ h3blk_config refiner_config(const h3blk_config& c) {
   return r;
 }
 
-ModelLayout model_layout(const h3blk_config& c, const h3blk_mod_weights& t, int64_t n, int64_t nt) {
+ModelLayout model_layout(const h3blk_config& c, const h3blk_mod_weights& t, int64_t n, int64_t nt, int keep) {
   ModelLayout L;
   std::memset(&L, 0, sizeof(L));
   const size_t C = c.hidden, N = (size_t)n, NT = (size_t)nt;
-  size_t blk = h3api::block_workspace_bytes(c, n);
+  size_t blk = h3api::block_workspace_bytes(c, n, keep);
   if (nt > 0) {
-    const size_t r = h3api::block_workspace_bytes(refiner_config(c), nt);
+    const size_t r = h3api::block_workspace_bytes(refiner_config(c), nt, keep);
     if (r > blk) blk = r;
   }
   size_t o = 0;
@@ -113,7 +113,7 @@ int check_forward(const h3blk_ctx* h, const h3blk_model_config* mc, const h3blk_
                         w->audio_out_w, w->refiner_gain};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return H3BLK_ERR_INVALID_ARG;
-  if (ws_bytes < model_layout(c, w->time, in->n_rows, in->n_text).total) return H3BLK_ERR_INVALID_ARG;
+  if (ws_bytes < model_layout(c, w->time, in->n_rows, in->n_text, h->keep_per_1024).total) return H3BLK_ERR_INVALID_ARG;
   return H3BLK_OK;
 }
 
@@ -132,7 +132,7 @@ int run_forward(const h3blk_ctx* h, const h3blk_model_config* mc, const h3blk_mo
   if (st != H3BLK_OK) return st;
   const h3blk_config& c = h->cfg;
   const int64_t N = in->n_rows, NT = in->n_text;
-  const ModelLayout L = model_layout(c, w->time, N, NT);
+  const ModelLayout L = model_layout(c, w->time, N, NT, h->keep_per_1024);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   int* err = reinterpret_cast<int*>(ws + L.block);  // the block workspace's error word
   auto* xa = reinterpret_cast<__nv_bfloat16*>(ws + L.xa);
@@ -277,7 +277,7 @@ int h3blk_model_workspace_bytes(h3blk_handle h, const h3blk_model_config* mc, co
   const int st = check_model(h, mc, time);
   if (st != H3BLK_OK) return st;
   if (!bytes || n_rows < 1 || n_text < 0 || n_text > n_rows) return H3BLK_ERR_INVALID_ARG;
-  *bytes = model_layout(h->cfg, *time, n_rows, n_text).total;
+  *bytes = model_layout(h->cfg, *time, n_rows, n_text, h->keep_per_1024).total;
   return H3BLK_OK;
 }
 

@@ -69,6 +69,7 @@ int check_group(const h3blk_ctx* h, int64_t n_rows, const h3blk_ulysses* u) {
   if (!h || !u || n_rows < 1) return H3BLK_ERR_INVALID_ARG;
   if (u->world < 1 || u->world > H3BLK_MAX_RANKS || u->rank < 0 || u->rank >= u->world) return H3BLK_ERR_INVALID_ARG;
   if (h->cfg.heads % u->world || n_rows % u->world) return H3BLK_ERR_UNSUPPORTED;
+  if (h->keep_per_1024 < 1024) return H3BLK_ERR_UNSUPPORTED;  // block-sparse attention is single-device
   return H3BLK_OK;
 }
 
@@ -77,7 +78,7 @@ h3api::BlockBufs bufs(const h3blk_ctx* h, int64_t n_rows, const h3blk_ulysses* u
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   auto at = [&](size_t off, bool used) { return used ? ws + off : nullptr; };
   const bool q = h->cfg.quant != 0;
-  h3api::BlockBufs b;
+  h3api::BlockBufs b{};  // sparse buffers and anything unset stay null
   b.err = reinterpret_cast<int*>(ws + L.err);
   b.tiles = reinterpret_cast<h3::TileInfo*>(ws + L.tiles);
   b.h1 = reinterpret_cast<__nv_bfloat16*>(at(L.h1, !q));

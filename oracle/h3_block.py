@@ -319,15 +319,19 @@ class BlockOracle:
             k_all[s:e], v_all[s:e] = kv["k"], kv["v"]
         return k_all, v_all
 
-    def query(self, x_rows, tag_rows, tidx_rows, pos_rows, table, k_all, v_all, doc_all):
+    def query(self, x_rows, tag_rows, tidx_rows, pos_rows, table, k_all, v_all, doc_all, o_given=None):
         """Every stage of the block for the given query rows, attending to
-        the keys / values of the whole sequence."""
+        the keys / values of the whole sequence (or taking the attention
+        output ``o_given`` [R, H, D] from another attention, e.g. block-sparse)."""
         d = self.d
         xr = f64(x_rows)
         m = modulation(f64(table), tag_rows, tidx_rows)
         h1 = adaln(xr, m[:, MOD_SHIFT1], m[:, MOD_SCALE1], d.norm_eps)
         q = self.qkv(h1, pos_rows, part=("q",))["q"]
-        o = attention(q, k_all, v_all, documents(tag_rows), doc_all).reshape(xr.shape[0], d.hd)
+        if o_given is None:
+            o = attention(q, k_all, v_all, documents(tag_rows), doc_all).reshape(xr.shape[0], d.hd)
+        else:
+            o = f64(o_given).reshape(xr.shape[0], d.hd)
         x1 = xr + m[:, MOD_GATE1] * self.linear(o, "o")
         h2 = adaln(x1, m[:, MOD_SHIFT2], m[:, MOD_SCALE2], d.norm_eps)
         g_u = self.linear(h2, "13")
@@ -335,10 +339,12 @@ class BlockOracle:
         out = x1 + m[:, MOD_GATE2] * self.linear(a, "2")
         return {"h1": h1, "q": q, "o": o, "x1": x1, "h2": h2, "a": a, "out": out}
 
-    def forward(self, x, tag, tidx, pos, table, rows=None, kv_chunk=4096):
+    def forward(self, x, tag, tidx, pos, table, rows=None, kv_chunk=4096, keep=None):
         """Block forward. ``rows`` (sorted indices) restricts every per-row
         stage to those query rows; k and v are always computed for all rows,
-        since every query sees every key of its document. Returns a dict of
+        since every query sees every key of its document. ``keep`` (bool
+        [blocks, heads, tiles]) replaces dense attention with block-sparse
+        attention over those tiles. Returns a dict of
         stages for the returned rows: h1, q, k, v, o, x1, h2, a, out (and the
         full-sequence k, v under "k_all", "v_all")."""
         x = f64(x)
@@ -348,6 +354,14 @@ class BlockOracle:
         N = x.shape[0]
         rows = np.arange(N) if rows is None else np.asarray(rows)
         k_all, v_all = self.kv_all(x, tag, tidx, pos, table, kv_chunk)
-        r = self.query(x[rows], tag[rows], tidx[rows], pos[rows], table, k_all, v_all, documents(tag))
+        o_given = None
+        if keep is not None:
+            # block-sparse attention (oracle/h3_sparse.py) with the given kept tiles
+            from .h3_sparse import sparse_attention
+            m = modulation(f64(table), tag, tidx)
+            h1 = adaln(x, m[:, MOD_SHIFT1], m[:, MOD_SCALE1], self.d.norm_eps)
+            q_all = self.qkv(h1, pos, part=("q",))["q"]
+            o_given = sparse_attention(q_all, k_all, v_all, tag, keep, rows=rows)[rows]
+        r = self.query(x[rows], tag[rows], tidx[rows], pos[rows], table, k_all, v_all, documents(tag), o_given)
         r.update({"rows": rows, "k": k_all[rows], "v": v_all[rows], "k_all": k_all, "v_all": v_all})
         return r

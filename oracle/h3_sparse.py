@@ -15,7 +15,8 @@ s1. The sequence is cut into key tiles of 128 rows and query blocks of 256
     valid (non-padding) rows, per head.
 s2. Score(block B, tile J, head h) = mean q_B,h . mean k_J,h. Candidate tiles
     are those with at least one valid row.
-s3. Each (block, head) keeps k = max(1, ceil(density x candidates)) tiles: the
+s3. Each (block, head) keeps k = max(1, ceil(n x m / 1024)) of its n
+    candidate tiles, m = round(1024 x density) (density in 1/1024 steps): the
     highest scores, ties broken toward the lower tile index. A block without
     valid rows keeps nothing (its rows are padding, whose attention output the
     block's zero gates discard).
@@ -63,7 +64,11 @@ def block_scores(q, k, tag):
 
 
 def keep_count(density, n_cand):
-    return max(1, math.ceil(density * n_cand)) if n_cand else 0
+    """k = max(1, ceil(n m / 1024)), m = round(1024 density), in integers."""
+    if not n_cand:
+        return 0
+    m = min(1024, max(1, int(round(1024.0 * density))))
+    return max(1, (n_cand * m + 1023) // 1024)
 
 
 def select(scores, cand, block_valid, density):
@@ -82,18 +87,20 @@ def select(scores, cand, block_valid, density):
     return keep
 
 
-def sparse_attention(q, k, v, tag, keep):
-    """Attention of every valid query row restricted to the valid keys of its
-    block's kept tiles. q, k, v: [N, H, D]; returns [N, H, D] (padding rows 0)."""
+def sparse_attention(q, k, v, tag, keep, rows=None):
+    """Attention of every valid query row (or of the given rows only)
+    restricted to the valid keys of its block's kept tiles. q, k, v:
+    [N, H, D]; returns [N, H, D] (rows not computed, and padding rows, 0)."""
     q, k, v = f64(q), f64(k), f64(v)
     N, H, D = q.shape
     valid = np.asarray(tag) != TAG_PAD
+    want = np.ones(N, dtype=bool) if rows is None else np.isin(np.arange(N), rows)
     out = np.zeros((N, H, D))
     scale = 1.0 / math.sqrt(D)
     tile_of = np.arange(N) // TILE
     for b in range(keep.shape[0]):
-        rows = np.arange(b * BLOCK, min(N, (b + 1) * BLOCK))
-        rows = rows[valid[rows]]
+        rows_b = np.arange(b * BLOCK, min(N, (b + 1) * BLOCK))
+        rows = rows_b[valid[rows_b] & want[rows_b]]
         if rows.size == 0:
             continue
         for h in range(H):

@@ -346,3 +346,22 @@ def test_ulysses_phases_validate_before_gpu(case, status):
         st_out = B.H3BLK_ERR_CUDA if case == "misaligned_peer" else status
         assert B.h3blk_ulysses_out(blk.handle, 320, u, p(10), p(11), p(12), p(14), w, p(15), p(20), ws,
                                    None) == st_out
+
+
+def test_attention_density_setting():
+    blk = j.H3Block(hi.TINY)
+    dense = blk.workspace_bytes(320)
+    for bad in (0.0, -0.5, 1.5, float("nan")):
+        assert B.h3blk_set_attention_density(blk.handle, bad) == B.H3BLK_ERR_INVALID_ARG
+    blk.set_attention_density(0.25)
+    sparse = blk.workspace_bytes(320)
+    n_tiles = 3
+    assert sparse >= dense + 2 * (n_tiles + 1) // 2 * 6 * (1 + n_tiles) * 4
+    off, nb = B.h3blk_stage_view(blk.handle, 320, "KV_LIST")
+    assert nb == 2 * 6 * (1 + n_tiles) * 4
+    # sequence parallelism is single-mode: block-sparse is refused there
+    with pytest.raises(B.H3BlkError) as e:
+        B.h3blk_ulysses_workspace_bytes(blk.handle, 320, 2)
+    assert e.value.status == B.H3BLK_ERR_UNSUPPORTED
+    blk.set_attention_density(1.0)
+    assert blk.workspace_bytes(320) == dense
