@@ -225,7 +225,7 @@ def measure_int8_peak(torch, device):
         return None
 
 
-def run_gpu_case(torch, j, hi, name, steps, warmup, device, peaks, int8_peak, clocks=None, e2e=False):
+def run_gpu_case(torch, j, hi, name, steps, warmup, device, peaks, int8_peak, clocks=None, e2e=False, density=1.0):
     from joint_video_audio_b200 import _binding as B
     dims, lay = hi.workload(name)
     inp = hi.make_inputs(dims, lay)
@@ -234,6 +234,8 @@ def run_gpu_case(torch, j, hi, name, steps, warmup, device, peaks, int8_peak, cl
     tag, tidx, pos = inp.tag.to(device), inp.tidx.to(device), inp.pos.to(device).contiguous()
     table = inp.table.to(device)
     blk = j.H3Block(dims)
+    if density < 1.0:
+        blk.set_attention_density(density)
     w = j.DeviceWeights.from_host(inp.weights, device)
     if dims.quant:
         w = blk.prepare_int8(w)
@@ -305,7 +307,18 @@ def run_gpu_case(torch, j, hi, name, steps, warmup, device, peaks, int8_peak, cl
            "seconds": secs_max, "ms_per_step": secs_max / steps * 1e3,
            "value": aggregate_throughput(n, steps, int(os.environ.get("WORLD_SIZE", "1")), secs_max),
            "kernels": kernels, "roofline": roof, "clocks": clk,
-           "gpu_launches": steps * (10 if dims.quant else 8)}
+           "gpu_launches": steps * ((10 if dims.quant else 8) + (2 if density < 1.0 else 0))}
+    if density < 1.0:
+        # work actually done: the kept (query tile, key tile) pairs
+        lists = blk.stage(ws, n, "KV_LIST")
+        kept = int(lists[:, :, 0].sum().item())
+        total = lists.shape[0] * lists.shape[1] * sum(1 for t in range(lists.shape[2] - 1)
+                                                       if lay.tag[t * 128:(t + 1) * 128].max() >= 0)
+        kept_flops = kept * 2 * 4 * 128 * 128 * dims.head_dim
+        a = kernels["attention"]
+        res["sparse"] = {"density": density, "kept_tile_fraction": kept / total,
+                         "attention_ms": a["ms"], "kept_tflops": kept_flops / (a["ms"] / 1e3) / 1e12,
+                         "dense_equivalent_tflops": a.get("tflops")}
     if e2e:
         res["e2e"] = run_e2e(torch, blk, inp, w, ws, steps, warmup, device)
     del ws, w, out, x
@@ -504,6 +517,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-model", action="store_true", help="skip the whole-model forward legs")
+    ap.add_argument("--no-sparse", action="store_true", help="skip the block-sparse attention leg")
     args = ap.parse_args()
     assert args.warmup >= 3 or args.impl == "reference", "at least 3 warm-up steps"
     ws_, rank, local = dist_env()
@@ -544,6 +558,12 @@ def main():
     if not args.no_w8a8:
         w8 = run_gpu_case(torch, j, hi, "w8a8_t2va_32k", args.steps, args.warmup, device, peaks, int8_peak)
     modt = run_modulation(torch, j, hi, device, peaks, args.steps)
+    sparse = None
+    if not args.no_sparse:
+        sp = run_gpu_case(torch, j, hi, args.workload, args.steps, args.warmup, device, peaks, int8_peak,
+                          density=0.25)
+        sparse = {"workload": sp["workload"], "value": sp["value"], "unit": UNIT, "ms_per_step": sp["ms_per_step"],
+                  **sp["sparse"], "gpu_launches": sp["gpu_launches"]}
     models = []
     if not args.no_model:
         for q in (0, 1):
@@ -572,6 +592,8 @@ def main():
         line["modulation_table"] = modt
         if models:
             line["model_forward"] = models
+        if sparse:
+            line["sparse_attention"] = sparse
         print(json.dumps(line), flush=True)
     import torch.distributed as dist
     if dist.is_initialized():
