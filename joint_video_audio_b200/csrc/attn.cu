@@ -309,30 +309,37 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         break;
       }
       tc_fence_after();
-      uint32_t u[kTile];
-      tmem_ld128(t_s, u);
-      float* sv = reinterpret_cast<float*>(u);
-      {
-        const int kk = tile_kind(ti);
-        if (!(kk == myk && myk != 2) || ti.rows < kTile) {
-          const int rows = ti.rows;
+      // S is read from tensor memory in 64-column halves, twice (once for the
+      // row max, once for the exponentials), so only 64 S values are live in
+      // registers at a time.
+      const int kk_kind = tile_kind(ti);
+      const bool need_mask = !(kk_kind == myk && myk != 2) || ti.rows < kTile;
+      auto mask_half = [&](float* sv, int h) {
+        if (!need_mask) return;
 #pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            const uint32_t bits = ti.padbits[w] ^ (my_pad ? 0xffffffffu : 0u);  // 1 = other document
+        for (int ww = 0; ww < 2; ++ww) {
+          const int w = 2 * h + ww;
+          const uint32_t bits = ti.padbits[w] ^ (my_pad ? 0xffffffffu : 0u);  // 1 = other document
 #pragma unroll
-            for (int c = 0; c < 32; ++c)
-              if (((bits >> c) & 1u) || w * 32 + c >= rows) sv[w * 32 + c] = -CUDART_INF_F;
-          }
+          for (int c = 0; c < 32; ++c)
+            if (((bits >> c) & 1u) || w * 32 + c >= ti.rows) sv[ww * 32 + c] = -CUDART_INF_F;
         }
-      }
+      };
       // row max: eight independent chains of three-input max
       float mc[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mc[i] = fmaxf(sv[2 * i], sv[2 * i + 1]);
+      for (int i = 0; i < 8; ++i) mc[i] = -CUDART_INF_F;
 #pragma unroll
-      for (int c = 16; c < kTile; c += 16)
+      for (int h = 0; h < 2; ++h) {
+        uint32_t u[64];
+        tmem_ld64(t_s + 64 * h, u);
+        float* sv = reinterpret_cast<float*>(u);
+        mask_half(sv, h);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) mc[i] = max3f(mc[i], sv[c + 2 * i], sv[c + 2 * i + 1]);
+        for (int c = 0; c < 64; c += 16)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mc[i] = max3f(mc[i], sv[c + 2 * i], sv[c + 2 * i + 1]);
+      }
       const float m8 = fmaxf(max3f(mc[0], mc[1], mc[2]), max3f(mc[3], mc[4], max3f(mc[5], mc[6], mc[7])));
       const float m_new = fmaxf(m_run, m8 * scale_log2);
       const bool grow = m_new > m_run + kRescaleThreshold || (m_run == -CUDART_INF_F && m_new != -CUDART_INF_F);
@@ -341,25 +348,30 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       const float alpha = grow ? ex2_approx(m_run - m_use) : 1.f;
       // exponentials on pairs: x = s * scale - m with one packed FMA; one pair
       // in kPolyEvery goes through the FMA-pipe polynomial, the rest through
-      // the MUFU, so both units share the load. P is packed to bf16 pairs in
-      // place (u[0..63]); the row sum runs in two packed accumulators. Each
-      // half of P (keys 0..63, then 64..127) is stored and announced on its
-      // own barrier, so the P V product starts on the first half while the
-      // second is computed.
+      // the MUFU, so both units share the load. Each half of P (keys 0..63,
+      // then 64..127) is packed to bf16 pairs, stored over the first 64
+      // columns of this tile's S and announced on its own barrier, so the
+      // P V product starts on the first half while the second is computed.
+      // The row sum runs in two packed accumulators.
       const uint64_t sc2 = f2_pack(scale_log2, scale_log2), nm2 = f2_pack(-m_sub, -m_sub);
       uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = acc0;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
+        uint32_t u[64];
+        tmem_ld64(t_s + 64 * h, u);
+        float* sv = reinterpret_cast<float*>(u);
+        mask_half(sv, h);
 #pragma unroll
-        for (int c = 64 * h; c < 64 * h + 64; c += 2) {
+        for (int c = 0; c < 64; c += 2) {
+          const int cg = 64 * h + c;  // column within the tile
           float x0, x1;
           f2_unpack(f2_fma(f2_pack(sv[c], sv[c + 1]), sc2, nm2), x0, x1);
           uint64_t e;
-          if (((c >> 1) % kPolyEvery) == kPolyEvery - 1)
+          if (((cg >> 1) % kPolyEvery) == kPolyEvery - 1)
             e = f2_exp2_poly(x0, x1);
           else
             e = f2_pack(ex2_approx(x0), ex2_approx(x1));
-          if ((c >> 1) & 1)
+          if ((cg >> 1) & 1)
             acc1 = f2_add(acc1, e);
           else
             acc0 = f2_add(acc0, e);
@@ -367,8 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
           f2_unpack(e, e0, e1);
           u[c >> 1] = pack_bf16x2(e0, e1);
         }
-        // P half -> tensor memory, over the first 64 columns of this tile's S
-        tmem_st32(t_s + 32 * h, *reinterpret_cast<const uint32_t(*)[32]>(u + 32 * h));
+        tmem_st32(t_s + 32 * h, *reinterpret_cast<const uint32_t(*)[32]>(u));
         if (h == 0 && j > 0 && __any_sync(0xffffffffu, grow)) {
           // O must be rescaled before the first P V step of this tile adds to
           // it; S_t of this tile completing implied the previous P V completed
