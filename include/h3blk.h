@@ -63,7 +63,7 @@ extern "C" {
 /* ------------------------------------------------------------------ status */
 #define H3BLK_OK 0
 #define H3BLK_ERR_INVALID_ARG 1 /* null / misaligned pointer, bad size, aliasing */
-#define H3BLK_ERR_UNSUPPORTED 2 /* a dimension this build does not handle */
+#define H3BLK_ERR_UNSUPPORTED 2 /* a dimension this library does not handle */
 #define H3BLK_ERR_CUDA 3        /* a CUDA runtime / driver call failed */
 #define H3BLK_ERR_TIMEOUT 4     /* a kernel pipeline wait gave up (reported by h3blk_check) */
 #define H3BLK_ERR_BAD_INDEX 5   /* a tag / timestep index outside the table (h3blk_check) */
