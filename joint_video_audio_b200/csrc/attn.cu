@@ -216,18 +216,36 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       constexpr uint32_t idesc_qk = make_idesc(1, 1, kTile, kTile, false);
       constexpr uint32_t idesc_pv = make_idesc(1, 1, kTile, D, true);
       const uint32_t q0 = smem_u32(s.q0), ring0 = smem_u32(s.slot0);
-      auto slot_of = [](int u) { return u % kSlots; };
-      auto wait_ring = [&](int u) { return mbar_wait(&s.ring_full[u % kSlots], (u / kSlots) & 1, abort); };
+      // ring position of load u = 2 j (K_j) or 2 j + 1 (V_j): slot u % kSlots,
+      // phase (u / kSlots) & 1, tracked incrementally (no division per step)
+      struct RingPos {
+        int slot;
+        uint32_t phase;
+        __device__ void advance(int by) {
+          slot += by;
+          while (slot >= kSlots) {
+            slot -= kSlots;
+            phase ^= 1u;
+          }
+        }
+      };
+      auto wait_ring = [&](const RingPos& r) { return mbar_wait(&s.ring_full[r.slot], r.phase, abort); };
       // S_t = Q_t K_j^T into TMEM columns [t*128, t*128+128)
-      auto issue_s = [&](int t, int j) -> bool {
+      // Shared-memory descriptors: the start-address field (bits 0..13, in
+      // 16-byte units) never carries out of its 14 bits inside shared memory,
+      // so a K step's descriptor is the tile's base descriptor plus a constant.
+      const uint64_t qdesc0 = sw128_desc(q0, 16);
+      const uint64_t ring_desc0 = sw128_desc(ring0, 16);
+      const uint64_t vdesc0 = sw128_desc(ring0, SM::kRegion);
+      auto issue_s = [&](int t, int kslot) -> bool {
         tc_fence_after();
-        const uint32_t qa = q0 + t * SM::kQBytes;
-        const uint32_t ka = ring0 + slot_of(2 * j) * SM::kKVBytes;
+        const uint64_t qd = qdesc0 + (uint64_t)((t * SM::kQBytes) >> 4);
+        const uint64_t kd = ring_desc0 + (uint64_t)((kslot * SM::kKVBytes) >> 4);
+        const uint32_t dtm = tmem + t * kTile;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * SM::kRegion + (kk & 3) * 32;
-          mma_bf16_ss(tmem + t * kTile, sw128_desc(qa + off, 16), sw128_desc(ka + off, 16), idesc_qk,
-                      kk > 0 ? 1u : 0u);
+          const uint64_t off = (uint64_t)(((kk >> 2) * SM::kRegion + (kk & 3) * 32) >> 4);
+          mma_bf16_ss(dtm, qd + off, kd + off, idesc_qk, kk > 0 ? 1u : 0u);
         }
         mma_commit(&s.s_full[t]);
         return true;
@@ -236,42 +254,45 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       // TMEM columns [t*128, t*128 + 64), 8 columns per K = 16 step
       // Each half of P (keys 0..63, 64..127) has its own ready barrier, so the
       // first four K steps run while the softmax still works on the second half.
-      auto issue_pv = [&](int t, int j) -> bool {
-        const uint32_t va = ring0 + slot_of(2 * j + 1) * SM::kKVBytes;
+      auto issue_pv = [&](int t, int j, int vslot) -> bool {
+        const uint64_t vd = vdesc0 + (uint64_t)((vslot * SM::kKVBytes) >> 4);
+        const uint32_t dtm = tmem + 256 + t * kTile, atm = tmem + t * kTile;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           if (!mbar_wait(half == 0 ? &s.p_lo[t] : &s.p_hi[t], j & 1, abort)) return false;
           tc_fence_after();
 #pragma unroll
-          for (int kk = 4 * half; kk < 4 * half + 4; ++kk) {
-            const uint64_t bd = sw128_desc(va + kk * 16 * 128, SM::kRegion);
-            mma_bf16_ts(tmem + 256 + t * kTile, tmem + t * kTile + kk * 8, bd, idesc_pv,
+          for (int kk = 4 * half; kk < 4 * half + 4; ++kk)
+            mma_bf16_ts(dtm, atm + kk * 8, vd + (uint64_t)((kk * 16 * 128) >> 4), idesc_pv,
                         (j > 0 || kk > 0) ? 1u : 0u);
-          }
         }
         return true;
       };
       bool ok = mbar_wait(s.q_full, 0, abort);
       if (ok && n_kv > 0) {
-        ok = wait_ring(0) && issue_s(0, 0) && issue_s(1, 0);
-        if (ok) mma_commit(&s.ring_empty[slot_of(0)]);
+        const RingPos k0{0, 0u};
+        ok = wait_ring(k0) && issue_s(0, 0) && issue_s(1, 0);
+        if (ok) mma_commit(&s.ring_empty[0]);
+        RingPos vpos{1, 0u}, kpos{2 % kSlots, 2 >= kSlots ? 1u : 0u};  // V_j and K_{j+1}
         for (int j = 0; ok && j < n_kv; ++j) {
           // the ring waits come first: they are normally satisfied long before
           // P, and polling them between P V and the next S would put their
           // latency on the critical path
           const bool more = j + 1 < n_kv;
-          ok = wait_ring(2 * j + 1) && (!more || wait_ring(2 * j + 2)) && issue_pv(0, j);
+          ok = wait_ring(vpos) && (!more || wait_ring(kpos)) && issue_pv(0, j, vpos.slot);
           if (!ok) break;
-          if (more) ok = issue_s(0, j + 1);
+          if (more) ok = issue_s(0, kpos.slot);
           if (!ok) break;
-          ok = issue_pv(1, j);
+          ok = issue_pv(1, j, vpos.slot);
           if (!ok) break;
-          mma_commit(&s.ring_empty[slot_of(2 * j + 1)]);
+          mma_commit(&s.ring_empty[vpos.slot]);
           if (more) {
-            ok = issue_s(1, j + 1);
+            ok = issue_s(1, kpos.slot);
             if (!ok) break;
-            mma_commit(&s.ring_empty[slot_of(2 * j + 2)]);
+            mma_commit(&s.ring_empty[kpos.slot]);
           }
+          vpos.advance(2);
+          kpos.advance(2);
         }
       }
       if (!ok) fail(p.err, abort);
