@@ -55,9 +55,11 @@ class H3Block:
 
     def __del__(self):
         h = getattr(self, "handle", None)
-        if h:
+        if h and B is not None and getattr(B, "h3blk_destroy", None) is not None:
+            # at interpreter exit the binding may already be torn down; the
+            # process exit then releases the handle
             B.h3blk_destroy(h)
-            self.handle = None
+        self.handle = None
 
     # ------------------------------------------------------------ attention mode
     def set_attention_density(self, density: float) -> None:

@@ -152,9 +152,9 @@ class ModelGraph:
 
     def __del__(self):
         h = getattr(self, "handle", None)
-        if h:
+        if h and B is not None and getattr(B, "h3blk_graph_destroy", None) is not None:
             B.h3blk_graph_destroy(h)
-            self.handle = None
+        self.handle = None
 
 
 __all__ = ["DeviceInputs", "DeviceModel", "Model", "ModelGraph"]
