@@ -122,6 +122,22 @@ __device__ __forceinline__ void load_chunk(uint32_t taddr, float sa, const float
   for (int j = 0; j < 32; ++j) v[j] = acc_value<INT8>(r[j], sa, sb, col + j);
 }
 
+// cos and sin of a rotary angle: the angle is reduced to [-pi, pi] by a
+// two-constant Cody-Waite step (Cody and Waite, "Software Manual for the
+// Elementary Functions", 1980: 2 pi split into its nearest float and the
+// remainder, each product taken exactly inside an FMA), then the hardware
+// sine / cosine, accurate to about 2^-21 on that interval. The angles are
+// position x frequency with positions of a few thousand at most.
+__device__ __forceinline__ void rope_sincos(float x, float& sn, float& cs) {
+  constexpr float kTwoPiHi = 6.28318548202514648f;   // float(2 pi)
+  constexpr float kTwoPiLo = -1.74845553146951e-07f;  // 2 pi - float(2 pi)
+  constexpr float kInvTwoPi = 0.159154943091895336f;
+  const float k = rintf(x * kInvTwoPi);
+  float r = fmaf(-k, kTwoPiHi, x);
+  r = fmaf(-k, kTwoPiLo, r);
+  __sincosf(r, &sn, &cs);
+}
+
 // ------------------------------------------------------------------ epilogue
 template <int EPI, bool INT8>
 __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tacc, int64_t row, bool row_ok, int n_tile,
@@ -264,7 +280,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tacc, 
           if (ax < 3) {
             float sn, cs;
             const int pv = ax == 0 ? pos3[0] : (ax == 1 ? pos3[1] : pos3[2]);
-            sincosf((float)pv * p.rope.freq[pair], &sn, &cs);
+            rope_sincos((float)pv * p.rope.freq[pair], sn, cs);
             const float a = v[2 * q], b = v[2 * q + 1];
             v[2 * q] = a * cs - b * sn;
             v[2 * q + 1] = a * sn + b * cs;
