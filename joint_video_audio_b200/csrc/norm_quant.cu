@@ -170,11 +170,12 @@ __device__ __forceinline__ void fwht128_chunk(float (&h)[8], int lane) {
   }
 #pragma unroll
   for (int m = 1; m < 16; m <<= 1) {
-    const bool upper = (lane & m) != 0;
+    // lower lane: h + other; upper lane: other - h (one FMA with a sign)
+    const float sgn = (lane & m) ? -1.f : 1.f;
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const float other = __shfl_xor_sync(0xffffffffu, h[e], m);
-      h[e] = upper ? (other - h[e]) : (h[e] + other);
+      h[e] = fmaf(sgn, h[e], other);
     }
   }
   const float inv_sqrt128 = 0.08838834764831845f;
@@ -197,16 +198,20 @@ __device__ __forceinline__ float block_reduce(float v, bool is_max, float* red) 
 // value instead of a division (the two can round a value lying within an ulp
 // of a half-integer differently, the int8 operand tolerance of the tests).
 __device__ __forceinline__ void quant_store(const float (&h)[8], float inv_s, bool zero, int8_t* dst) {
-  uint32_t w[2] = {0u, 0u};
+  uint32_t w[2];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    int q = 0;
-    if (!zero) {
-      float t = rintf(h[e] * inv_s);
-      t = fminf(fmaxf(t, -127.f), 127.f);
-      q = (int)t;
+  for (int g = 0; g < 2; ++g) {
+    int q[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      // round to nearest even, then clamp (|h| <= amax keeps it within 127)
+      const int v = zero ? 0 : __float2int_rn(h[4 * g + e] * inv_s);
+      q[e] = max(-127, min(127, v));
     }
-    w[e >> 2] |= (uint32_t)(q & 0xff) << (8 * (e & 3));
+    // bytes 0..3 from the low bytes of q[0..3]
+    const uint32_t lo = __byte_perm((uint32_t)q[0], (uint32_t)q[1], 0x0040);
+    const uint32_t hi = __byte_perm((uint32_t)q[2], (uint32_t)q[3], 0x0040);
+    w[g] = __byte_perm(lo, hi, 0x5410);
   }
   *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
 }
