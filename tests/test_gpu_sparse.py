@@ -102,3 +102,25 @@ def test_real_dims_sparse_sampled_rows():
     o_ref = sparse_attention(q, k, v, lay.tag, keep, rows=rows)[rows]
     o_gpu = case.stage("O")[torch.from_numpy(rows).cuda()].float().cpu().numpy().reshape(len(rows), d.heads, d.head_dim)
     assert_intermediate("o", o_gpu, o_ref)
+
+
+def test_padded_32k_sparse_sampled_rows():
+    """The 32k layout with 168 padding rows at the tail: padding tiles are
+    never candidates, mixed tiles are masked per key, padding rows pass the
+    block through unchanged."""
+    inp = hi.make_inputs("t2va_32k_pad168")
+    case = GpuCase(inp)
+    case.block.set_attention_density(0.3)
+    case.ws = case.block.workspace(case.n)
+    case.run()
+    assert case.block.check(case.ws, case.n) == 0
+    lay, d = inp.layout, inp.dims
+    q, k, v = _qkv64(case, d)
+    keep = _gpu_keep(case, lay.n)
+    _check_selection(keep, q, k, lay.tag, 0.3)
+    rows = hi.sample_rows(lay, k=32, k_pad=0, seed=4)
+    o_ref = sparse_attention(q, k, v, lay.tag, keep, rows=rows)[rows]
+    o_gpu = case.stage("O")[torch.from_numpy(rows).cuda()].float().cpu().numpy().reshape(len(rows), d.heads, d.head_dim)
+    assert_intermediate("o", o_gpu, o_ref)
+    pad = torch.from_numpy(lay.tag == -1).cuda()
+    assert torch.equal(case.out[pad], case.x[pad])
