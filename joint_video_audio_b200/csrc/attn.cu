@@ -47,6 +47,27 @@
 namespace h3 {
 namespace {
 
+// 64 consecutive 32-bit columns of the warp's 32 lanes, without the wait:
+// the registers are valid only after tcgen05.wait::ld.
+__device__ __forceinline__ void tmem_ld64_nowait(uint32_t taddr, uint32_t (&r)[64]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+      "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+        "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
+        "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
+        "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
 constexpr int kTile = 128;
 constexpr int kSoftmaxWarps = 8;
 constexpr int kThreads = 32 * (2 + kSoftmaxWarps);
@@ -317,14 +338,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     bool ok = true;
     int j = 0;
     int kt = seq.at(0, -1);
-    TileInfo ti_next;
-    if (kt < n_tiles) ti_next = p.tiles[kt];
     for (; kt < n_tiles; ++j) {
-      const TileInfo ti = ti_next;
-      // the next KV tile's summary is fetched before waiting for S, so its
-      // global-memory latency hides behind the wait
+      // the tile summary is fetched before waiting for S, so its global-memory
+      // latency hides behind the wait
+      const int4 tiw0 = __ldg(reinterpret_cast<const int4*>(p.tiles + kt));
+      const int2 tiw1 = __ldg(reinterpret_cast<const int2*>(p.tiles + kt) + 2);
       const int kt_next = seq.at(j + 1, kt);
-      if (kt_next < n_tiles) ti_next = p.tiles[kt_next];
       if (!mbar_wait(&s.s_full[t], j & 1, abort)) {
         ok = false;
         break;
@@ -333,6 +352,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       // S is read from tensor memory in 64-column halves, twice (once for the
       // row max, once for the exponentials), so only 64 S values are live in
       // registers at a time.
+      TileInfo ti;
+      ti.rows = tiw0.x;
+      ti.npad = tiw0.y;
+      ti.padbits[0] = (uint32_t)tiw0.z;
+      ti.padbits[1] = (uint32_t)tiw0.w;
+      ti.padbits[2] = (uint32_t)tiw1.x;
+      ti.padbits[3] = (uint32_t)tiw1.y;
       const int kk_kind = tile_kind(ti);
       const bool need_mask = !(kk_kind == myk && myk != 2) || ti.rows < kTile;
       auto mask_half = [&](float* sv, int h) {
@@ -346,16 +372,28 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             if (((bits >> c) & 1u) || w * 32 + c >= ti.rows) sv[ww * 32 + c] = -CUDART_INF_F;
         }
       };
-      // row max: eight independent chains of three-input max
+      // S in two 64-column halves: the second half's load is in flight while
+      // the first half's max is taken; both stay in registers for the
+      // exponentials (one read of S per tile)
+      uint32_t u0[64], u1[64];
+      tmem_ld64_nowait(t_s, u0);
+      tmem_wait_ld();
+      tmem_ld64_nowait(t_s + 64, u1);
       float mc[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) mc[i] = -CUDART_INF_F;
+      {
+        float* sv = reinterpret_cast<float*>(u0);
+        mask_half(sv, 0);
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t u[64];
-        tmem_ld64(t_s + 64 * h, u);
-        float* sv = reinterpret_cast<float*>(u);
-        mask_half(sv, h);
+        for (int c = 0; c < 64; c += 16)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mc[i] = max3f(mc[i], sv[c + 2 * i], sv[c + 2 * i + 1]);
+      }
+      tmem_wait_ld();
+      {
+        float* sv = reinterpret_cast<float*>(u1);
+        mask_half(sv, 1);
 #pragma unroll
         for (int c = 0; c < 64; c += 16)
 #pragma unroll
@@ -378,10 +416,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = acc0;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        uint32_t u[64];
-        tmem_ld64(t_s + 64 * h, u);
+        uint32_t* u = h == 0 ? u0 : u1;
         float* sv = reinterpret_cast<float*>(u);
-        mask_half(sv, h);
 #pragma unroll
         for (int c = 0; c < 64; c += 2) {
           const int cg = 64 * h + c;  // column within the tile
