@@ -233,6 +233,7 @@ int phase_qkv(const h3blk_ctx* h, const Span& sp, const void* x, const int32_t* 
   mn.out_bf16 = b.h1;
   if (q) mn.out_bf16 = nullptr;
   H3_TRY(mark(h, timing, 1, s));
+  mn.err = b.err;
   H3_TRY(h3::launch_modnorm(mn, s));
 
   // ---- QKV projection + QK-RMSNorm + RoPE (optionally routed by head group)
@@ -318,7 +319,7 @@ int phase_out(const h3blk_ctx* h, const Span& sp, const void* x, const int32_t* 
   const int32_t* ti = tidx + sp.row0;
 
   // ---- out-projection + gated residual
-  if (q) H3_TRY(h3::launch_rotate_quant(b.o, n, (int)HD, b.o_q, b.o_s, s));
+  if (q) H3_TRY(h3::launch_rotate_quant(b.o, n, (int)HD, b.o_q, b.o_s, b.err, s));
   GemmArgs g = base_gemm(h, b.err);
   g.A = q ? (const void*)b.o_q : (const void*)b.o;
   g.B = w->wo;
@@ -357,6 +358,7 @@ int phase_out(const h3blk_ctx* h, const Span& sp, const void* x, const int32_t* 
   mn.out_q = b.h2_q;
   mn.out_scale = b.h2_s;
   mn.out_bf16 = q ? nullptr : b.h2;
+  mn.err = b.err;
   H3_TRY(h3::launch_modnorm(mn, s));
 
   // ---- FFN up (W1 | W3) + SwiGLU
@@ -377,7 +379,7 @@ int phase_out(const h3blk_ctx* h, const Span& sp, const void* x, const int32_t* 
   H3_TRY(mark(h, timing, 8, s));
 
   // ---- FFN down + gated residual
-  if (q) H3_TRY(h3::launch_rotate_quant(b.a, n, (int)F, b.a_q, b.a_s, s));
+  if (q) H3_TRY(h3::launch_rotate_quant(b.a, n, (int)F, b.a_q, b.a_s, b.err, s));
   g = base_gemm(h, b.err);
   g.A = q ? (const void*)b.a_q : (const void*)b.a;
   g.B = w->w2;
@@ -573,7 +575,7 @@ int h3blk_check(h3blk_handle h, int64_t n_rows, const void* workspace, void* str
   if (cudaMemcpy(&bits, static_cast<const uint8_t*>(workspace) + L.off[H3BLK_STAGE_ERROR], sizeof(int),
                  cudaMemcpyDeviceToHost) != cudaSuccess)
     return H3BLK_ERR_CUDA;
-  if (bits & (h3::kErrTimeoutGemm | h3::kErrTimeoutAttn))
+  if (bits & (h3::kErrTimeoutGemm | h3::kErrTimeoutAttn | h3::kErrTimeoutStream))
     *status = H3BLK_ERR_TIMEOUT;
   else if (bits & (h3::kErrBadIndex | h3::kErrBadRowIndex))
     *status = H3BLK_ERR_BAD_INDEX;
@@ -607,7 +609,7 @@ int h3blk_prepare_int8_weights(h3blk_handle h, const h3blk_weights* in, void* bl
   const int64_t C = c.hidden, HD = (int64_t)c.heads * c.head_dim, F = c.ffn;
   auto rq = [&](const void* w, int64_t rows, int K, size_t qo, size_t so) {
     return h3::launch_rotate_quant(static_cast<const __nv_bfloat16*>(w), rows, K,
-                                   reinterpret_cast<int8_t*>(bl + qo), reinterpret_cast<float*>(bl + so), s);
+                                   reinterpret_cast<int8_t*>(bl + qo), reinterpret_cast<float*>(bl + so), nullptr, s);
   };
   if (rq(in->wqkv, 3 * HD, (int)C, b.wqkv, b.s_qkv) != cudaSuccess) return H3BLK_ERR_CUDA;
   if (rq(in->wo, C, (int)HD, b.wo, b.s_o) != cudaSuccess) return H3BLK_ERR_CUDA;
@@ -695,7 +697,7 @@ int h3blk_rotate_quantize(int64_t rows, int K, const void* in_bf16, int8_t* out_
   int st = device_info(&sms, &enc);
   if (st != H3BLK_OK) return st;
   return cuda_status(h3::launch_rotate_quant(static_cast<const __nv_bfloat16*>(in_bf16), rows, K, out_q, out_scale,
-                                             reinterpret_cast<cudaStream_t>(stream)));
+                                             nullptr, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 static int plain_gemm(int64_t M, int N, int K, const void* A, const void* B, void* C, void* stream, bool int8) {

@@ -47,6 +47,7 @@ struct ModNormArgs {
   __nv_bfloat16* out_bf16;  // used when out_q == nullptr
   int8_t* out_q;
   float* out_scale;
+  int* err = nullptr;  // device error word (a load that never landed), may be null
 };
 cudaError_t launch_modnorm(const ModNormArgs& a, cudaStream_t s);
 
@@ -54,7 +55,7 @@ cudaError_t launch_modnorm(const ModNormArgs& a, cudaStream_t s);
 // Rows of a bf16 matrix [rows, K] -> block-128 Hadamard rotation ->
 // symmetric per-row int8 with fp32 scale.
 cudaError_t launch_rotate_quant(const __nv_bfloat16* in, int64_t rows, int K, int8_t* out_q, float* out_scale,
-                                cudaStream_t s);
+                                int* err, cudaStream_t s);
 
 // ---------------------------------------------------------------- GEMM
 enum GemmEpilogue : int {

@@ -294,7 +294,7 @@ int h3blk_model_check(const void* workspace, void* stream, int* status) {
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return H3BLK_ERR_CUDA;
   int bits = 0;
   if (cudaMemcpy(&bits, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return H3BLK_ERR_CUDA;
-  if (bits & (h3::kErrTimeoutGemm | h3::kErrTimeoutAttn))
+  if (bits & (h3::kErrTimeoutGemm | h3::kErrTimeoutAttn | h3::kErrTimeoutStream))
     *status = H3BLK_ERR_TIMEOUT;
   else if (bits & (h3::kErrBadIndex | h3::kErrBadRowIndex))
     *status = H3BLK_ERR_BAD_INDEX;

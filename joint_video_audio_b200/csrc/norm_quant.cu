@@ -91,65 +91,6 @@ __device__ __forceinline__ const float* mod_row(const float* table, const int32_
   return table + ((int64_t)tg * n_t + ti) * 6 * C;
 }
 
-// ============================================================== K1 (bf16)
-// One warp per row; lane l owns the 16-byte chunks l, l+32, l+64, ...
-constexpr int kModNormMaxChunksPerLane = 24;  // hidden <= 6144
-
-__global__ void __launch_bounds__(256) modnorm_bf16_kernel(ModNormArgs a) {
-  const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (row >= a.n) return;
-  const int lane = threadIdx.x & 31;
-  const int nchunk = a.C >> 3;
-  const uint4* xr = reinterpret_cast<const uint4*>(a.x + row * a.C);
-  uint4 v[kModNormMaxChunksPerLane];
-  float ss = 0.f;
-#pragma unroll
-  for (int i = 0; i < kModNormMaxChunksPerLane; ++i) {
-    const int c = lane + 32 * i;
-    if (c < nchunk) {
-      v[i] = ld_nc_v4(xr + c);
-      float f[8];
-      bf16x8_to_f32(v[i], f);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
-    }
-  }
-  ss = warp_sum(ss);
-  const float rstd = rsqrtf(ss / (float)a.C + a.eps);
-  const float* m = mod_row(a.table, a.tag, a.tidx, row, a.n_tags, a.n_t, a.C);
-  const float* shift = m ? m + (int64_t)a.shift_idx * a.C : nullptr;
-  const float* scale = m ? m + (int64_t)a.scale_idx * a.C : nullptr;
-  uint4* outr = reinterpret_cast<uint4*>(a.out_bf16 + row * a.C);
-#pragma unroll
-  for (int i = 0; i < kModNormMaxChunksPerLane; ++i) {
-    const int c = lane + 32 * i;
-    if (c < nchunk) {
-      float f[8];
-      bf16x8_to_f32(v[i], f);
-      float sh[8], sc[8];
-      if (m) {
-        const float4* s4 = reinterpret_cast<const float4*>(shift + c * 8);
-        const float4* k4 = reinterpret_cast<const float4*>(scale + c * 8);
-        float4 s0 = __ldg(s4), s1 = __ldg(s4 + 1), k0 = __ldg(k4), k1 = __ldg(k4 + 1);
-        sh[0] = s0.x; sh[1] = s0.y; sh[2] = s0.z; sh[3] = s0.w; sh[4] = s1.x; sh[5] = s1.y; sh[6] = s1.z; sh[7] = s1.w;
-        sc[0] = k0.x; sc[1] = k0.y; sc[2] = k0.z; sc[3] = k0.w; sc[4] = k1.x; sc[5] = k1.y; sc[6] = k1.z; sc[7] = k1.w;
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) sh[e] = sc[e] = 0.f;
-      }
-      float h[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) h[e] = fmaf(f[e] * rstd, 1.f + sc[e], sh[e]);
-      uint4 o;
-      o.x = pack_bf16x2(h[0], h[1]);
-      o.y = pack_bf16x2(h[2], h[3]);
-      o.z = pack_bf16x2(h[4], h[5]);
-      o.w = pack_bf16x2(h[6], h[7]);
-      outr[c] = o;
-    }
-  }
-}
-
 // ============================================================== rotation + quant
 // One CTA per row at a time; thread t owns chunks t, t + THREADS, ... of 8
 // channels (THREADS a multiple of 16). A 128-channel Hadamard block is 16
@@ -320,8 +261,172 @@ static cudaError_t launch_rq(const __nv_bfloat16* in, int64_t rows, int K, int8_
   }
 }
 
+// ============================================================== K1 (bf16), row streaming
+// h = rmsnorm(x)(1 + scale) + shift, stored as bf16: a pass bound by moving
+// each row in and out once. Persistent CTAs walk the rows (row = blockIdx.x +
+// k * gridDim.x); each row reaches shared memory by one bulk copy (TMA
+// engine), issued `stages` rows ahead into a ring, so every CTA keeps several
+// rows in flight while its threads work on one. Thread t owns the 16-byte
+// chunks t, t + THREADS, ... of the row (8 channels each).
+constexpr int kMaxStages = 8;
+constexpr int kStageBudget = 48 * 1024;  // shared-memory bytes of one CTA's ring
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+// Modulation vectors of one chunk (zero without a table row).
+__device__ __forceinline__ void mod_chunk(const float* m, const ModNormArgs& a, int K, int c, float (&sh)[8],
+                                          float (&sc)[8]) {
+  if (m) {
+    const float4* s4 = reinterpret_cast<const float4*>(m + (int64_t)a.shift_idx * K + c * 8);
+    const float4* k4 = reinterpret_cast<const float4*>(m + (int64_t)a.scale_idx * K + c * 8);
+    const float4 s0 = __ldg(s4), s1 = __ldg(s4 + 1), k0 = __ldg(k4), k1 = __ldg(k4 + 1);
+    sh[0] = s0.x; sh[1] = s0.y; sh[2] = s0.z; sh[3] = s0.w; sh[4] = s1.x; sh[5] = s1.y; sh[6] = s1.z; sh[7] = s1.w;
+    sc[0] = k0.x; sc[1] = k0.y; sc[2] = k0.z; sc[3] = k0.w; sc[4] = k1.x; sc[5] = k1.y; sc[6] = k1.z; sc[7] = k1.w;
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) sh[e] = sc[e] = 0.f;
+  }
+}
+
+template <int CPT, int THREADS>
+__global__ void __launch_bounds__(THREADS) modnorm_stream_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows,
+                                                                 int K, int stages, __nv_bfloat16* __restrict__ out_h,
+                                                                 ModNormArgs a, int* err) {
+  extern __shared__ __align__(128) uint8_t ring[];
+  __shared__ uint64_t full[kMaxStages];
+  __shared__ float red[THREADS / 32];
+  const int nchunk = K >> 3;
+  const uint32_t row_bytes = (uint32_t)K * 2u;
+  const int64_t step = gridDim.x;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < stages; ++i) mbar_init(&full[i], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // load k of this CTA (row blockIdx.x + k * step) goes to stage k % stages
+  auto issue = [&](int64_t k) {
+    const int64_t row = blockIdx.x + k * step;
+    if (row >= rows) return;
+    const int st = (int)(k % stages);
+    mbar_expect_tx(&full[st], row_bytes);
+    bulk_load(ring + (size_t)st * row_bytes, in + row * (int64_t)K, row_bytes, &full[st]);
+  };
+  if (threadIdx.x == 0)
+    for (int k = 0; k < stages; ++k) issue(k);
+  for (int64_t k = 0;; ++k) {
+    const int64_t row = blockIdx.x + k * step;
+    if (row >= rows) break;
+    const int st = (int)(k % stages);
+    const bool ok = mbar_wait(&full[st], (uint32_t)((k / stages) & 1), nullptr);
+    float h[CPT][8];
+    const uint4* src = reinterpret_cast<const uint4*>(ring + (size_t)st * row_bytes);
+#pragma unroll
+    for (int i = 0; i < CPT; ++i) {
+      const int c = threadIdx.x + THREADS * i;
+      if (ok && c < nchunk) {
+        bf16x8_to_f32(src[c], h[i]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) h[i][e] = 0.f;
+      }
+    }
+    // every thread has its chunks in registers: the stage is refilled with
+    // the row `stages` steps ahead (or the CTA stops if a load never landed)
+    if (__syncthreads_or(!ok)) {
+      if (threadIdx.x == 0) {
+        if (err) atomicOr(err, kErrTimeoutStream);
+        // loads still in flight must land before the CTA's shared memory goes
+        for (int64_t kk = k; kk < k + stages && blockIdx.x + kk * step < rows; ++kk)
+          mbar_wait(&full[kk % stages], (uint32_t)((kk / stages) & 1), nullptr);
+      }
+      return;
+    }
+    if (threadIdx.x == 0) {
+      fence_proxy_async_smem();
+      issue(k + stages);
+    }
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < CPT; ++i)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ss = fmaf(h[i][e], h[i][e], ss);
+    ss = block_reduce(ss, false, red);
+    const float rstd = rsqrtf(ss / (float)K + a.eps);
+    const float* m = mod_row(a.table, a.tag, a.tidx, row, a.n_tags, a.n_t, K);
+    uint4* dst = reinterpret_cast<uint4*>(out_h + row * (int64_t)K);
+#pragma unroll
+    for (int i = 0; i < CPT; ++i) {
+      const int c = threadIdx.x + THREADS * i;
+      if (c < nchunk) {
+        float sh[8], sc[8];
+        mod_chunk(m, a, K, c, sh, sc);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) h[i][e] = fmaf(h[i][e] * rstd, 1.f + sc[e], sh[e]);
+        uint4 o;
+        o.x = pack_bf16x2(h[i][0], h[i][1]);
+        o.y = pack_bf16x2(h[i][2], h[i][3]);
+        o.z = pack_bf16x2(h[i][4], h[i][5]);
+        o.w = pack_bf16x2(h[i][6], h[i][7]);
+        dst[c] = o;
+      }
+    }
+  }
+}
+
+template <int CPT, int THREADS>
+static cudaError_t launch_rows_t(const __nv_bfloat16* in, int64_t rows, int K, __nv_bfloat16* out_h,
+                                 const ModNormArgs& a, int* err, cudaStream_t s) {
+  auto kern = modnorm_stream_kernel<CPT, THREADS>;
+  const size_t row_bytes = (size_t)K * 2;
+  int stages = (int)(kStageBudget / row_bytes);
+  stages = stages < 2 ? 2 : (stages > kMaxStages ? kMaxStages : stages);
+  const size_t smem = (size_t)stages * row_bytes;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 0, per_sm = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, THREADS, smem)) != cudaSuccess) return e;
+  if (per_sm < 1) per_sm = 1;
+  const int64_t grid = rows < (int64_t)sms * per_sm ? rows : (int64_t)sms * per_sm;
+  kern<<<(unsigned)grid, THREADS, smem, s>>>(in, rows, K, stages, out_h, a, err);
+  return cudaGetLastError();
+}
+
+// Thread count and chunks per thread for a row of K channels: exact fits for
+// the block's widths, otherwise 256 threads with enough chunks each.
+static cudaError_t launch_rows(const __nv_bfloat16* in, int64_t rows, int K, __nv_bfloat16* out_h, const ModNormArgs& a,
+                               int* err, cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
+  if (K <= 0 || K % 128 != 0) return cudaErrorInvalidValue;  // 16-byte rows, whole chunks per thread
+  const int nchunk = K / 8;
+#define H3_ROWS(CPT, T) return launch_rows_t<CPT, T>(in, rows, K, out_h, a, err, s)
+  if (nchunk == 672) H3_ROWS(3, 224);   // 5376 channels
+  if (nchunk == 896) H3_ROWS(4, 224);   // 7168
+  if (nchunk == 1792) H3_ROWS(7, 256);  // 14336
+  if (nchunk <= 32) H3_ROWS(1, 32);
+  if (nchunk <= 128) H3_ROWS(1, 128);
+  switch ((nchunk + 255) / 256) {
+    case 1: H3_ROWS(1, 256);
+    case 2: H3_ROWS(2, 256);
+    case 3: H3_ROWS(3, 256);
+    case 4: H3_ROWS(4, 256);
+    case 5: H3_ROWS(5, 256);
+    case 6: H3_ROWS(6, 256);
+    case 7: H3_ROWS(7, 256);
+    case 8: H3_ROWS(8, 256);
+    default:
+      return cudaErrorInvalidValue;
+  }
+#undef H3_ROWS
+}
+
 cudaError_t launch_rotate_quant(const __nv_bfloat16* in, int64_t rows, int K, int8_t* out_q, float* out_scale,
-                                cudaStream_t s) {
+                                int* /*err: this pass has no waits*/, cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
   ModNormArgs none{};
   return launch_rq<false>(in, rows, K, out_q, out_scale, none, s);
@@ -330,11 +435,7 @@ cudaError_t launch_rotate_quant(const __nv_bfloat16* in, int64_t rows, int K, in
 cudaError_t launch_modnorm(const ModNormArgs& a, cudaStream_t s) {
   if (a.n <= 0) return cudaSuccess;
   if (a.out_q) return launch_rq<true>(a.x, a.n, a.C, a.out_q, a.out_scale, a, s);
-  if (a.C / 8 > 32 * kModNormMaxChunksPerLane) return cudaErrorInvalidValue;
-  const int warps = 8;
-  const unsigned blocks = (unsigned)((a.n + warps - 1) / warps);
-  modnorm_bf16_kernel<<<blocks, warps * 32, 0, s>>>(a);
-  return cudaGetLastError();
+  return launch_rows(a.x, a.n, a.C, a.out_bf16, a, a.err, s);
 }
 
 }  // namespace h3

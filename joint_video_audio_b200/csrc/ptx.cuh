@@ -15,6 +15,7 @@ enum : int {
   kErrTimeoutGemm = 2,    // a GEMM pipeline wait ran out of time
   kErrTimeoutAttn = 4,    // an attention pipeline wait ran out of time
   kErrBadRowIndex = 8,    // a row index of the model shell outside the packed sequence
+  kErrTimeoutStream = 16, // a row-streaming load (norm / quantisation pass) never landed
 };
 
 // Wall-clock budget of a single pipeline wait before it is declared stuck.
