@@ -436,6 +436,17 @@ H3BLK_API int h3blk_attention_noalloc(int64_t n_rows, int heads, int head_dim, i
                                       const void* qkv, const int32_t* tag, const int32_t* tidx, void* o,
                                       void* stream);
 
+/* Test-only: runs, on `stream`, one bounded wait of the kind every pipeline
+ * wait of this library is (an mbarrier phase polled against a time limit), on
+ * a barrier whose phase completes first (complete != 0) or never completes
+ * (complete == 0), with a limit of limit_ms milliseconds (1..2000). It then
+ * synchronises `stream` and sets *status to what h3blk_check reports for the
+ * outcome: H3BLK_OK, or H3BLK_ERR_TIMEOUT when the wait ran out. The kernel
+ * returns normally either way, so the CUDA context stays usable. `word` is a
+ * caller-owned device int32 (4-byte aligned) used as the error word; it is
+ * reset by the call. INVALID_ARG for a null pointer or a limit out of range. */
+H3BLK_API int h3blk_selftest_wait(int complete, int limit_ms, void* word, void* stream, int* status);
+
 /* Message for a status code (static storage). */
 H3BLK_API const char* h3blk_error_string(int status);
 

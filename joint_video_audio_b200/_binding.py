@@ -31,7 +31,8 @@ EXPORTS = ["h3blk_create", "h3blk_destroy", "h3blk_workspace_bytes", "h3blk_stag
            "h3blk_modulation_table", "h3blk_model_workspace_bytes", "h3blk_model_forward", "h3blk_model_check",
            "h3blk_model_graph_create", "h3blk_graph_launch", "h3blk_graph_info", "h3blk_graph_destroy",
            "h3blk_ulysses_buffer_bytes", "h3blk_ulysses_workspace_bytes", "h3blk_ulysses_qkv",
-           "h3blk_ulysses_attention", "h3blk_ulysses_out", "h3blk_set_attention_density"]
+           "h3blk_ulysses_attention", "h3blk_ulysses_out", "h3blk_set_attention_density",
+           "h3blk_selftest_wait"]
 
 H3BLK_MAX_RANKS = 8
 
@@ -119,6 +120,7 @@ def _load():
         "h3blk_version": (i32, []),
         "h3blk_set_kernel_events": (i32, [vp, C.POINTER(vp), i32]),
         "h3blk_attention_noalloc": (i32, [i64, i32, i32, i32, i32, vp, vp, vp, vp, vp]),
+        "h3blk_selftest_wait": (i32, [i32, i32, vp, vp, C.POINTER(i32)]),
         "h3blk_modulation_scratch_bytes": (i32, [vp, C.POINTER(h3blk_mod_weights), C.POINTER(sz)]),
         "h3blk_modulation_table": (i32, [vp, C.POINTER(h3blk_mod_weights), C.POINTER(C.c_float),
                                           C.POINTER(C.c_float), C.c_float, vp, vp, sz, vp]),
@@ -253,6 +255,15 @@ def h3blk_attention_noalloc(n_rows, heads, head_dim, n_tags, n_t, qkv, tag, tidx
     """Raw call (pointers are ints); returns the status code. Uses the
     library's fixed device scratch instead of a caller workspace."""
     return _lib.h3blk_attention_noalloc(n_rows, heads, head_dim, n_tags, n_t, qkv, tag, tidx, o, stream)
+
+
+def h3blk_selftest_wait(complete: bool, limit_ms: int, word, stream) -> int:
+    """Test-only: one bounded pipeline wait on a barrier that completes
+    (complete=True) or never does; returns the status h3blk_check would give
+    (H3BLK_OK or H3BLK_ERR_TIMEOUT). `word` is a device int32 pointer."""
+    st = C.c_int32()
+    _check("h3blk_selftest_wait", _lib.h3blk_selftest_wait(1 if complete else 0, limit_ms, word, stream, C.byref(st)))
+    return st.value
 
 
 def h3blk_modulation_scratch_bytes(handle, w: h3blk_mod_weights) -> int:

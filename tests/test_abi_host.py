@@ -365,3 +365,10 @@ def test_attention_density_setting():
     assert e.value.status == B.H3BLK_ERR_UNSUPPORTED
     blk.set_attention_density(1.0)
     assert blk.workspace_bytes(320) == dense
+
+
+@pytest.mark.parametrize("limit_ms,word", [(0, 256), (2001, 256), (50, 0), (50, 258)])
+def test_selftest_wait_validates_before_gpu(limit_ms, word):
+    st = C.c_int32()
+    rc = B._lib.h3blk_selftest_wait(0, limit_ms, word, None, C.byref(st))
+    assert rc == B.H3BLK_ERR_INVALID_ARG
