@@ -4,6 +4,8 @@ decision taken from fp32 pooled scores on the GPU: every kept tile must be
 among the oracle's best within a small score margin (ties may go either way),
 and the attention and block outputs are then compared with the GPU's own
 selection."""
+from dataclasses import replace
+
 import numpy as np
 import pytest
 import torch
@@ -51,9 +53,10 @@ def _qkv64(case, d):
     return q.double().numpy(), k.double().numpy(), v.double().numpy()
 
 
-@pytest.mark.parametrize("density", [0.34, 0.5])
-def test_tiny_sparse_block(density):
-    inp = hi.make_inputs("tiny_320")
+@pytest.mark.parametrize("density,quant", [(0.34, 0), (0.5, 0), (0.34, 1)])
+def test_tiny_sparse_block(density, quant):
+    dims, lay = hi.workload("tiny_320")
+    inp = hi.make_inputs(replace(dims, quant=quant), lay)
     case = GpuCase(inp)
     case.block.set_attention_density(density)
     case.ws = case.block.workspace(case.n)
