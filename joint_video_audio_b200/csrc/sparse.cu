@@ -11,8 +11,8 @@
 // density in 1/1024 units. A block without valid rows keeps its own first
 // tile (its rows are padding; their attention output is discarded).
 //
-// Two kernels: per (tile, head) sums of q and k over valid rows (one thread
-// per channel, rows read as coalesced 256-byte lines), then per (block, head)
+// Two kernels: per (tile, channel) sums of q and k over valid rows (16-byte
+// loads, each row read as coalesced 2 KB runs), then per (block, head)
 // the scores against every tile, the rank of each candidate, and the kept
 // tiles written in ascending order as [count, tile, tile, ...].
 #include <cuda_bf16.h>
@@ -26,27 +26,59 @@ namespace {
 constexpr int kTileRows = 128;
 constexpr int kSelThreads = 256;
 
-// sums[(tile * H + h) * D + d] over valid rows of q (part 0) and k (part 1)
-__global__ void pool_kernel(const __nv_bfloat16* __restrict__ qkv, const int32_t* __restrict__ tag, int64_t n,
-                            int heads, int D, float* __restrict__ qsum, float* __restrict__ ksum,
-                            int32_t* __restrict__ count) {
-  const int tile = blockIdx.x, h = blockIdx.y, d = threadIdx.x;
-  const int64_t HD = (int64_t)heads * D, ld = 3 * HD;
+// Sums over a tile's valid rows of q and k, stored as [tile][heads][head_dim]
+// (= tile * HD + channel). One CTA per (128-row tile, 1024-channel window):
+// threads 0..127 own 16-byte chunks of the window's q channels, threads
+// 128..255 the same chunks of k, so each row is read as two coalesced 2 KB
+// runs; four rows are loaded before any is added, keeping several loads in
+// flight per thread.
+constexpr int kPoolThreads = 256;
+constexpr int kPoolWindow = 1024;  // channels per CTA (128 chunks of 8)
+constexpr int kPoolUnroll = 4;
+
+__global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __nv_bfloat16* __restrict__ qkv,
+                                                             const int32_t* __restrict__ tag, int64_t n, int HD,
+                                                             float* __restrict__ qsum, float* __restrict__ ksum,
+                                                             int32_t* __restrict__ count) {
+  const int tile = blockIdx.x, part = threadIdx.x >> 7;  // part 0: q, 1: k
+  const int c = blockIdx.y * kPoolWindow + (threadIdx.x & 127) * 8;  // first channel of the chunk
+  const int64_t ld = 3 * (int64_t)HD;
   const int64_t r0 = (int64_t)tile * kTileRows;
-  const int64_t r1 = r0 + kTileRows < n ? r0 + kTileRows : n;
-  float sq = 0.f, sk = 0.f;
-  int c = 0;
-  for (int64_t r = r0; r < r1; ++r) {
-    if (__ldg(tag + r) == -1) continue;
-    const __nv_bfloat16* row = qkv + r * ld + (int64_t)h * D + d;
-    sq += __bfloat162float(row[0]);
-    sk += __bfloat162float(row[HD]);
-    ++c;
+  const int rows = (int)(r0 + kTileRows < n ? kTileRows : n - r0);
+  const bool on = c < HD;
+  const __nv_bfloat16* src = qkv + r0 * ld + (int64_t)part * HD + (on ? c : 0);
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+  int valid = 0;
+  for (int r = 0; r < rows; r += kPoolUnroll) {
+    uint4 v[kPoolUnroll];
+    bool use[kPoolUnroll];
+#pragma unroll
+    for (int u = 0; u < kPoolUnroll; ++u) {
+      use[u] = r + u < rows && __ldg(tag + r0 + r + u) != -1;
+      if (on && use[u]) v[u] = __ldg(reinterpret_cast<const uint4*>(src + (int64_t)(r + u) * ld));
+    }
+#pragma unroll
+    for (int u = 0; u < kPoolUnroll; ++u) {
+      if (!use[u]) continue;
+      ++valid;
+      if (!on) continue;
+      const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+        acc[2 * i] += f.x;
+        acc[2 * i + 1] += f.y;
+      }
+    }
   }
-  const int64_t o = ((int64_t)tile * heads + h) * D + d;
-  qsum[o] = sq;
-  ksum[o] = sk;
-  if (h == 0 && d == 0) count[tile] = c;
+  if (on) {
+    float4* dst = reinterpret_cast<float4*>((part ? ksum : qsum) + (int64_t)tile * HD + c);
+    dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+  }
+  if (blockIdx.y == 0 && threadIdx.x == 0) count[tile] = valid;
 }
 
 // one CTA per (query block, head)
@@ -137,8 +169,10 @@ cudaError_t launch_sparse_select(const SparseArgs& a, cudaStream_t s) {
   const int n_tiles = (int)((a.n + kTileRows - 1) / kTileRows);
   const int n_blocks = (n_tiles + 1) / 2;
   if (a.head_dim > 256 || a.keep_per_1024 < 1 || a.keep_per_1024 > 1024) return cudaErrorInvalidValue;
-  pool_kernel<<<dim3((unsigned)n_tiles, (unsigned)a.heads), a.head_dim, 0, s>>>(a.qkv, a.tag, a.n, a.heads,
-                                                                              a.head_dim, a.qsum, a.ksum, a.count);
+  const int HD = a.heads * a.head_dim;
+  if (HD % 8 != 0) return cudaErrorInvalidValue;  // whole 16-byte chunks
+  pool_kernel<<<dim3((unsigned)n_tiles, (unsigned)((HD + kPoolWindow - 1) / kPoolWindow)), kPoolThreads, 0, s>>>(
+      a.qkv, a.tag, a.n, HD, a.qsum, a.ksum, a.count);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const size_t smem = (size_t)a.head_dim * 4 + (size_t)n_tiles * 8;
