@@ -6,8 +6,9 @@
 // wait simply returns false after its time limit.
 #include <cuda_runtime.h>
 
+#include <cstdint>
+
 #include "../../include/h3blk.h"
-#include "api_internal.h"
 #include "ptx.cuh"
 
 namespace {
