@@ -372,3 +372,19 @@ def test_selftest_wait_validates_before_gpu(limit_ms, word):
     st = C.c_int32()
     rc = B._lib.h3blk_selftest_wait(0, limit_ms, word, None, C.byref(st))
     assert rc == B.H3BLK_ERR_INVALID_ARG
+
+
+def test_block_sparse_mode_sizes_block_and_model_workspaces():
+    """Block-sparse attention needs its pooled sums and kept-tile lists in the
+    workspace: the block's and the model's sizes both grow with the mode, and
+    density 1 is dense again."""
+    blk = j.H3Block(hi.TINY)
+    mc, w, _, _ = _fake_model()
+    dense_blk = blk.workspace_bytes(320)
+    dense_model = B.h3blk_model_workspace_bytes(blk.handle, mc, w.time, 320, 64)
+    blk.set_attention_density(0.3)
+    assert blk.workspace_bytes(320) > dense_blk
+    assert B.h3blk_model_workspace_bytes(blk.handle, mc, w.time, 320, 64) > dense_model
+    blk.set_attention_density(1.0)
+    assert blk.workspace_bytes(320) == dense_blk
+    assert B.h3blk_model_workspace_bytes(blk.handle, mc, w.time, 320, 64) == dense_model
