@@ -438,3 +438,114 @@ def test_gate1_gates_attention_and_gate2_gates_ffn(tiny):
     r3 = _fwd(ob, inp, table=t3)
     np.testing.assert_array_equal(r3["x1"], _fwd(ob, inp)["x1"])
     assert not np.allclose(r3["out"], _fwd(ob, inp)["out"])
+
+
+# ---------------------------------------------------------------------------
+# Readings pinned by hand values: which coordinate drives which rotary pair
+# block, and which half of the SwiGLU weight goes through silu. Each pin is a
+# function so that the planted-mistake tests below can show that it catches a
+# swapped copy of the oracle.
+# ---------------------------------------------------------------------------
+
+def _rope_axis_pin():
+    # rope_pairs (1, 2, 1), head_dim 8: pair 0 follows t, pairs 1-2 follow h,
+    # pair 3 follows w. Frequencies: t [1], h [1, 1e4^(-1/2) = 0.01], w [1].
+    # Input pairs (1,2) (3,4) (5,6) (7,8); a pair (a, b) turned by phi becomes
+    # (a cos phi - b sin phi, a sin phi + b cos phi).
+    x = np.arange(1.0, 9.0).reshape(1, 1, 8)
+    c, s = math.cos, math.sin
+    cases = {
+        (0, 1, 0): [1, 2, 3 * c(1) - 4 * s(1), 3 * s(1) + 4 * c(1),
+                    5 * c(0.01) - 6 * s(0.01), 5 * s(0.01) + 6 * c(0.01), 7, 8],
+        (0, 3, 0): [1, 2, 3 * c(3) - 4 * s(3), 3 * s(3) + 4 * c(3),
+                    5 * c(0.03) - 6 * s(0.03), 5 * s(0.03) + 6 * c(0.03), 7, 8],
+        (0, 0, 1): [1, 2, 3, 4, 5, 6, 7 * c(1) - 8 * s(1), 7 * s(1) + 8 * c(1)],
+        (1, 0, 0): [1 * c(1) - 2 * s(1), 1 * s(1) + 2 * c(1), 3, 4, 5, 6, 7, 8],
+        (2, 0, 5): [1 * c(2) - 2 * s(2), 1 * s(2) + 2 * c(2), 3, 4, 5, 6,
+                    7 * c(5) - 8 * s(5), 7 * s(5) + 8 * c(5)],
+    }
+    for p, want in cases.items():
+        got = orc.apply_rope(x, np.array([p]), (1, 2, 1), 1e4)
+        np.testing.assert_allclose(got[0, 0], want, atol=1e-12, err_msg=f"position {p}")
+
+
+def test_rope_axis_to_pair_block_mapping_hand_values():
+    _rope_axis_pin()
+
+
+def _swiglu_half_pin():
+    # C = 4, F = 1, H = 1, D = 6. gate1 = 0 so x1 = x; gate2 = 1. x = [1, 2, 0, 0]
+    # with eps 0 gives h2 = x / sqrt(5/4) = [2/sqrt5, 4/sqrt5, 0, 0].
+    # w13 row 0 (the W1 half, through silu) reads h2[0]; row 1 (the W3 half,
+    # the linear "up" branch) reads h2[1]: a = silu(2/sqrt5) * 4/sqrt5.
+    dims = SimpleNamespace(hidden=4, heads=1, head_dim=6, ffn=1, hd=6, n_tags=1, n_t=1,
+                           rope_pairs=(1, 1, 1), rope_theta=10000.0, norm_eps=0.0,
+                           qk_norm_eps=1e-6, quant=0)   # q = k = 0 here; eps keeps their norm finite
+    w13 = np.zeros((2, 4)); w13[0, 0] = 1.0; w13[1, 1] = 1.0
+    w2 = np.zeros((4, 1)); w2[0, 0] = 1.0
+    w = SimpleNamespace(wqkv=np.zeros((18, 4)), q_gain=np.ones(6), k_gain=np.ones(6),
+                        wo=np.zeros((4, 6)), w13=w13, w2=w2)
+    table = np.zeros((1, 1, 6, 4))
+    table[0, 0, orc.MOD_GATE2] = 1.0
+    x = np.array([[1.0, 2.0, 0.0, 0.0]])
+    r = orc.BlockOracle(dims, w).forward(x, np.array([0]), np.array([0]), np.array([[0, 0, 0]]), table)
+    g, u = 2 / math.sqrt(5), 4 / math.sqrt(5)
+    a = g / (1 + math.exp(-g)) * u          # 1.1357...; the swapped reading gives 1.3709...
+    np.testing.assert_allclose(r["a"][0], [a], atol=1e-12)
+    np.testing.assert_allclose(r["out"][0], [1 + a, 2, 0, 0], atol=1e-12)
+
+
+def test_swiglu_w1_half_goes_through_silu_hand_values():
+    _swiglu_half_pin()
+
+
+def test_swiglu_hand_value_with_distinct_gate_and_up():
+    # silu(2) * 3 = 3 * 2 / (1 + e^-2); silu(3) * 2 would be 5.7155...
+    np.testing.assert_allclose(orc.swiglu(np.array([2.0]), np.array([3.0])), [6 / (1 + math.exp(-2))], rtol=1e-15)
+
+
+# Planted mistakes (in the oracle, on the CPU): each pin above must fail on a
+# plausibly wrong copy of the function it guards.
+
+def _rope_angles_axes_swapped(pos, rope_pairs, theta, head_dim):
+    pos = np.asarray(pos, dtype=np.float64)[:, [0, 2, 1]]       # h and w exchanged
+    return _ORIG_ROPE_ANGLES(pos, rope_pairs, theta, head_dim)
+
+
+def _rope_angles_axes_reversed(pos, rope_pairs, theta, head_dim):
+    pos = np.asarray(pos, dtype=np.float64)[:, ::-1]             # pos[:, 2 - axis]
+    return _ORIG_ROPE_ANGLES(pos, rope_pairs, theta, head_dim)
+
+
+def _rope_angles_doubled_exponent(pos, rope_pairs, theta, head_dim):
+    pos = np.asarray(pos, dtype=np.float64)
+    ang = np.zeros((pos.shape[0], head_dim // 2))
+    j = 0
+    for axis, n in enumerate(rope_pairs):
+        ang[:, j:j + n] = pos[:, axis:axis + 1] * theta ** (-2.0 * np.arange(n) / n)
+        j += n
+    return ang
+
+
+_ORIG_ROPE_ANGLES = orc.rope_angles
+
+
+@pytest.mark.parametrize("mutant", [_rope_angles_axes_swapped, _rope_angles_axes_reversed,
+                                    _rope_angles_doubled_exponent])
+def test_rope_axis_pin_catches_planted_mistakes(monkeypatch, mutant):
+    monkeypatch.setattr(orc, "rope_angles", mutant)
+    with pytest.raises(AssertionError):
+        _rope_axis_pin()
+
+
+def test_rope_axis_pin_catches_a_flipped_rotation_sign(monkeypatch):
+    orig = orc.rope_angles
+    monkeypatch.setattr(orc, "rope_angles", lambda *a: -orig(*a))
+    with pytest.raises(AssertionError):
+        _rope_axis_pin()
+
+
+def test_swiglu_pin_catches_swapped_halves(monkeypatch):
+    monkeypatch.setattr(orc, "swiglu", lambda g, u: orc.silu(u) * g)
+    with pytest.raises(AssertionError):
+        _swiglu_half_pin()
