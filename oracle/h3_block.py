@@ -231,8 +231,19 @@ def quantize_rows(v):
 
 
 def int8_matmul_exact(a_q, w_q):
-    """Exact integer product acc[r, c] = sum_k a_q[r, k] * w_q[c, k] (int64)."""
-    return np.matmul(np.asarray(a_q, dtype=np.int64), np.asarray(w_q, dtype=np.int64).T)
+    """Exact integer product acc[r, c] = sum_k a_q[r, k] * w_q[c, k] (int64).
+
+    Computed as a float64 matrix product: every term is an integer of
+    magnitude <= 127 * 127, so every partial sum, in any order, is an integer
+    below 127^2 K < 2^53 and is represented exactly; the result is then the
+    exact integer sum (asserted bound on K)."""
+    a = np.asarray(a_q)
+    w = np.asarray(w_q)
+    K = a.shape[-1]
+    assert 127 * 127 * K < 2 ** 53
+    assert np.abs(a).max(initial=0) <= 127 and np.abs(w).max(initial=0) <= 127
+    acc = np.matmul(a.astype(np.float64), w.astype(np.float64).T)
+    return np.rint(acc).astype(np.int64)
 
 
 def prepare_int8_weight(w):
@@ -249,6 +260,14 @@ def w8a8_linear(a, wq, sw):
     return acc.astype(np.float64) * sa[:, None] * sw[None, :]
 
 
+def bf16_round(x):
+    """Round to the nearest bfloat16 value (ties to even), returned as float64.
+    Used only by the faithful mode of the block oracle."""
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float64))
+    return t.to(torch.bfloat16).to(torch.float64).numpy()
+
+
 # --------------------------------------------------------------------------
 # The block
 # --------------------------------------------------------------------------
@@ -260,10 +279,17 @@ class BlockOracle:
     norm_eps, qk_norm_eps and quant. ``weights`` carries bf16 wqkv [3HD, C],
     q_gain/k_gain [D], wo [C, HD], w13 [2F, C] (W1 rows then W3 rows) and
     w2 [C, F].
+
+    ``faithful=True`` is a diagnostic, not the contract: it rounds to bf16 at
+    the points where the block's stages are stored as bf16 (h1 and h2 on the
+    bf16 path, q, k, v, o, x1, a and out on both), so that a difference
+    against the GPU can be told apart from the rounding of those stores. The
+    default computes every stage in fp64 with no intermediate rounding.
     """
 
-    def __init__(self, dims, weights):
+    def __init__(self, dims, weights, faithful=False):
         self.d = dims
+        self.faithful = bool(faithful)
         self.quant = int(getattr(dims, "quant", 0))
         self.wqkv = f64(weights.wqkv)
         self.q_gain = f64(weights.q_gain)
@@ -275,12 +301,26 @@ class BlockOracle:
             self.int8 = {name: prepare_int8_weight(w) for name, w in
                          (("qkv", self.wqkv), ("o", self.wo), ("13", self.w13), ("2", self.w2))}
 
-    # linear y = a W^T, bf16 weights or rotated W8A8
-    def linear(self, a, name):
+    def _store(self, a):
+        """A stage as the block stores it: bf16 in faithful mode, else as is."""
+        return bf16_round(a) if self.faithful else a
+
+    def _store_bf16_path(self, a):
+        """h1 / h2: stored as bf16 on the bf16 path only (the W8A8 path
+        quantises them straight from fp32)."""
+        return bf16_round(a) if (self.faithful and not self.quant) else a
+
+    # linear y = a W^T, bf16 weights or rotated W8A8; ``rows`` selects output
+    # channels (weight rows), which leaves every computed column unchanged
+    def linear(self, a, name, rows=None):
         if self.quant:
             wq, sw = self.int8[name]
+            if rows is not None:
+                wq, sw = wq[rows], sw[rows]
             return w8a8_linear(a, wq, sw)
         w = {"qkv": self.wqkv, "o": self.wo, "13": self.w13, "2": self.w2}[name]
+        if rows is not None:
+            w = w[rows]
         return np.matmul(a, w.T)
 
     def _split_heads(self, y):
@@ -291,16 +331,20 @@ class BlockOracle:
         [R, H, D] arrays for the requested parts."""
         d = self.d
         HD = d.hd
-        y = self.linear(h1, "qkv")
+        names = [p for p in ("q", "k", "v") if p in part]
+        idx = {"q": 0, "k": 1, "v": 2}
+        cols = np.concatenate([np.arange(idx[p] * HD, (idx[p] + 1) * HD) for p in names])
+        y = self.linear(h1, "qkv", rows=None if len(names) == 3 else cols)
+        ys = {p: y[:, i * HD:(i + 1) * HD] for i, p in enumerate(names)}
         out = {}
         if "q" in part:
-            q = qk_rmsnorm(self._split_heads(y[:, :HD]), self.q_gain, d.qk_norm_eps)
-            out["q"] = apply_rope(q, pos, d.rope_pairs, d.rope_theta)
+            q = qk_rmsnorm(self._split_heads(ys["q"]), self.q_gain, d.qk_norm_eps)
+            out["q"] = self._store(apply_rope(q, pos, d.rope_pairs, d.rope_theta))
         if "k" in part:
-            k = qk_rmsnorm(self._split_heads(y[:, HD:2 * HD]), self.k_gain, d.qk_norm_eps)
-            out["k"] = apply_rope(k, pos, d.rope_pairs, d.rope_theta)
+            k = qk_rmsnorm(self._split_heads(ys["k"]), self.k_gain, d.qk_norm_eps)
+            out["k"] = self._store(apply_rope(k, pos, d.rope_pairs, d.rope_theta))
         if "v" in part:
-            out["v"] = self._split_heads(y[:, 2 * HD:])
+            out["v"] = self._store(self._split_heads(ys["v"]))
         return out
 
     def kv_all(self, x, tag, tidx, pos, table, kv_chunk=4096):
@@ -314,7 +358,7 @@ class BlockOracle:
         for s in range(0, N, kv_chunk):
             e = min(N, s + kv_chunk)
             m = modulation(table, tag[s:e], tidx[s:e])
-            h = adaln(x[s:e], m[:, MOD_SHIFT1], m[:, MOD_SCALE1], d.norm_eps)
+            h = self._store_bf16_path(adaln(x[s:e], m[:, MOD_SHIFT1], m[:, MOD_SCALE1], d.norm_eps))
             kv = self.qkv(h, pos[s:e], part=("k", "v"))
             k_all[s:e], v_all[s:e] = kv["k"], kv["v"]
         return k_all, v_all
@@ -326,17 +370,18 @@ class BlockOracle:
         d = self.d
         xr = f64(x_rows)
         m = modulation(f64(table), tag_rows, tidx_rows)
-        h1 = adaln(xr, m[:, MOD_SHIFT1], m[:, MOD_SCALE1], d.norm_eps)
+        h1 = self._store_bf16_path(adaln(xr, m[:, MOD_SHIFT1], m[:, MOD_SCALE1], d.norm_eps))
         q = self.qkv(h1, pos_rows, part=("q",))["q"]
         if o_given is None:
             o = attention(q, k_all, v_all, documents(tag_rows), doc_all).reshape(xr.shape[0], d.hd)
         else:
             o = f64(o_given).reshape(xr.shape[0], d.hd)
-        x1 = xr + m[:, MOD_GATE1] * self.linear(o, "o")
-        h2 = adaln(x1, m[:, MOD_SHIFT2], m[:, MOD_SCALE2], d.norm_eps)
+        o = self._store(o)
+        x1 = self._store(xr + m[:, MOD_GATE1] * self.linear(o, "o"))
+        h2 = self._store_bf16_path(adaln(x1, m[:, MOD_SHIFT2], m[:, MOD_SCALE2], d.norm_eps))
         g_u = self.linear(h2, "13")
-        a = swiglu(g_u[:, :d.ffn], g_u[:, d.ffn:])
-        out = x1 + m[:, MOD_GATE2] * self.linear(a, "2")
+        a = self._store(swiglu(g_u[:, :d.ffn], g_u[:, d.ffn:]))
+        out = self._store(x1 + m[:, MOD_GATE2] * self.linear(a, "2"))
         return {"h1": h1, "q": q, "o": o, "x1": x1, "h2": h2, "a": a, "out": out}
 
     def forward(self, x, tag, tidx, pos, table, rows=None, kv_chunk=4096, keep=None):
@@ -359,7 +404,7 @@ class BlockOracle:
             # block-sparse attention (oracle/h3_sparse.py) with the given kept tiles
             from .h3_sparse import sparse_attention
             m = modulation(f64(table), tag, tidx)
-            h1 = adaln(x, m[:, MOD_SHIFT1], m[:, MOD_SCALE1], self.d.norm_eps)
+            h1 = self._store_bf16_path(adaln(x, m[:, MOD_SHIFT1], m[:, MOD_SCALE1], self.d.norm_eps))
             q_all = self.qkv(h1, pos, part=("q",))["q"]
             o_given = sparse_attention(q_all, k_all, v_all, tag, keep, rows=rows)[rows]
         r = self.query(x[rows], tag[rows], tidx[rows], pos[rows], table, k_all, v_all, documents(tag), o_given)

@@ -549,3 +549,78 @@ def test_swiglu_pin_catches_swapped_halves(monkeypatch):
     monkeypatch.setattr(orc, "swiglu", lambda g, u: orc.silu(u) * g)
     with pytest.raises(AssertionError):
         _swiglu_half_pin()
+
+
+# ---------------------------------------------------------------------------
+# Faithful (bf16-store) diagnostic mode and the exact int8 product
+# ---------------------------------------------------------------------------
+
+def test_bf16_round_hand_values():
+    # bf16 keeps 8 significant bits: the spacing just above 1 is 2^-7
+    cases = [(1 + 2 ** -8, 1.0),                          # tie -> even (1.0)
+             (1 + 3 * 2 ** -8, 1 + 2 ** -6),              # tie -> even (mantissa 2)
+             (1 + 2 ** -8 + 2 ** -20, 1 + 2 ** -7),       # just above the tie
+             (-3.0, -3.0), (0.0, 0.0), (2 ** -130, 2 ** -130),
+             (65280.0 + 127.0, 65280.0), (255.0, 255.0), (257.0, 256.0), (259.0, 260.0)]
+    for v, want in cases:
+        assert orc.bf16_round(np.array([v]))[0] == want, v
+
+
+def test_faithful_mode_rounds_exactly_the_stored_stages(tiny):
+    inp, _ = tiny
+    lay = inp.layout
+    exact = orc.BlockOracle(inp.dims, inp.weights)
+    faith = orc.BlockOracle(inp.dims, inp.weights, faithful=True)
+    re_ = _fwd(exact, inp)
+    rf = _fwd(faith, inp)
+    for key in ("h1", "q", "k", "v", "o", "x1", "h2", "a", "out"):
+        np.testing.assert_array_equal(orc.bf16_round(rf[key]), rf[key], err_msg=key)
+    # the roundings move the output by a few bf16 ulps at most, never more
+    d = np.abs(rf["out"] - re_["out"])
+    assert d.max() < 4 * 2.0 ** -7 * max(1.0, np.abs(re_["out"]).max())
+    assert d.max() > 0
+    # zero gates: the identity survives the roundings (x is bf16 already)
+    table = inp.table.clone()
+    table[:, :, orc.MOD_GATE1] = 0
+    table[:, :, orc.MOD_GATE2] = 0
+    r0 = faith.forward(inp.x, lay.tag, lay.tidx, lay.pos, table)
+    np.testing.assert_array_equal(r0["out"], orc.f64(inp.x))
+
+
+def test_faithful_w8a8_leaves_the_quantised_inputs_unrounded(tiny):
+    inp, _ = tiny
+    faith = orc.BlockOracle(replace(inp.dims, quant=1), inp.weights, faithful=True)
+    r = _fwd(faith, inp, rows=np.arange(8))
+    # h1 feeds the rotation + quantisation straight from fp32 on this path
+    assert not np.array_equal(orc.bf16_round(r["h1"]), r["h1"])
+    np.testing.assert_array_equal(orc.bf16_round(r["o"]), r["o"])
+
+
+def test_int8_product_exact_at_extremes_and_random():
+    rng = np.random.default_rng(40)
+    a = rng.integers(-127, 128, size=(5, 14336)).astype(np.int8)
+    w = rng.integers(-127, 128, size=(3, 14336)).astype(np.int8)
+    got = orc.int8_matmul_exact(a, w)
+    for i in range(5):
+        for j in range(3):
+            assert got[i, j] == sum(int(p) * int(q) for p, q in zip(a[i].tolist(), w[j].tolist()))
+    full = np.full((1, 14336), 127, np.int8)
+    assert orc.int8_matmul_exact(full, full)[0, 0] == 127 * 127 * 14336
+    assert orc.int8_matmul_exact(full, -full)[0, 0] == -127 * 127 * 14336
+
+
+def test_qkv_parts_equal_the_full_projection(tiny):
+    inp, ob = tiny
+    lay = inp.layout
+    rng = np.random.default_rng(41)
+    h = rng.standard_normal((6, inp.dims.hidden))
+    pos = lay.pos[:6]
+    full = ob.qkv(h, pos)
+    kv = ob.qkv(h, pos, part=("k", "v"))
+    q = ob.qkv(h, pos, part=("q",))
+    np.testing.assert_array_equal(kv["k"], full["k"])
+    np.testing.assert_array_equal(kv["v"], full["v"])
+    np.testing.assert_array_equal(q["q"], full["q"])
+    obq = orc.BlockOracle(replace(inp.dims, quant=1), inp.weights)
+    fq = obq.qkv(h, pos)
+    np.testing.assert_array_equal(obq.qkv(h, pos, part=("k", "v"))["v"], fq["v"])
