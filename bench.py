@@ -219,16 +219,47 @@ def measure_int8_peak(torch, device):
             e.synchronize()
             best = min(best, s.elapsed_time(e) / 1e3)
         del a, b
-        return 2.0 * 8192 ** 3 / best / 1e12
+        return {"tops": 2.0 * 8192 ** 3 / best / 1e12,
+                "source": "int8 burst: torch._int_mm 8192^3, best of 10, measured in this run"}
     except Exception as ex:  # noqa: BLE001
         print(f"int8 peak measurement failed: {ex}", file=sys.stderr)
         return None
 
 
-def run_gpu_case(torch, j, hi, name, steps, warmup, device, peaks, int8_peak, clocks=None, e2e=False, density=1.0):
+class WeightCache:
+    """Host and device copies of the block weights, drawn once per weight
+    shape (every real-dimension workload shares them: same dims, same seed)."""
+
+    def __init__(self, torch, j, hi, device):
+        self.torch, self.j, self.hi, self.device = torch, j, hi, device
+        self.host, self.dev = {}, {}
+
+    @staticmethod
+    def _key(dims):
+        return (dims.hidden, dims.heads, dims.head_dim, dims.ffn)
+
+    def inputs(self, dims, lay):
+        k = self._key(dims)
+        if k not in self.host:
+            self.host[k] = self.hi.make_weights(dims)
+        return self.hi.Inputs(dims, lay, self.hi.make_x(dims, lay.n), self.hi.make_table(dims), self.host[k])
+
+    def device_weights(self, inp, blk):
+        k = self._key(inp.dims) + (int(inp.dims.quant),)
+        if k not in self.dev:
+            if k[:4] + (0,) not in self.dev:
+                self.dev[k[:4] + (0,)] = self.j.DeviceWeights.from_host(inp.weights, self.device)
+            if inp.dims.quant:
+                self.dev[k] = blk.prepare_int8(self.dev[k[:4] + (0,)])
+        return self.dev[k]
+
+
+def run_gpu_case(torch, j, hi, name, steps, warmup, device, peaks, int8_peak, clocks=None, e2e=False, density=1.0,
+                 cache=None):
     from joint_video_audio_b200 import _binding as B
     dims, lay = hi.workload(name)
-    inp = hi.make_inputs(dims, lay)
+    cache = cache or WeightCache(torch, j, hi, device)
+    inp = cache.inputs(dims, lay)
     n = lay.n
     x = inp.x.to(device)
     tag, tidx, pos = inp.tag.to(device), inp.tidx.to(device), inp.pos.to(device).contiguous()
@@ -236,9 +267,7 @@ def run_gpu_case(torch, j, hi, name, steps, warmup, device, peaks, int8_peak, cl
     blk = j.H3Block(dims)
     if density < 1.0:
         blk.set_attention_density(density)
-    w = j.DeviceWeights.from_host(inp.weights, device)
-    if dims.quant:
-        w = blk.prepare_int8(w)
+    w = cache.device_weights(inp, blk)
     ws = blk.workspace(n, device)
     out = torch.empty_like(x)
     stream = torch.cuda.current_stream(device)
@@ -281,12 +310,18 @@ def run_gpu_case(torch, j, hi, name, steps, warmup, device, peaks, int8_peak, cl
     fl = gemm_flops(dims, n)
     fl["attention"] = attention_flops(dims, lay)
     bt = hbm_bytes(dims, n, dims.quant)
-    tens_peak = peaks["bf16_tflops_sustained"]
+    # Kernels are timed one launch at a time inside a step of tens of
+    # milliseconds, so the burst peaks apply; the sustained bf16 fraction is
+    # kept beside them.
+    tens_peak = peaks["bf16_tflops"]
+    i8_peak = int8_peak["tops"] if int8_peak else None
     for nm, v in kernels.items():
         if nm in fl and v["ms"] > 0:
             v["tflops"] = fl[nm] / (v["ms"] / 1e3) / 1e12
-            p = (int8_peak if (dims.quant and nm != "attention") else tens_peak)
+            p = (i8_peak if (dims.quant and nm != "attention") else tens_peak)
             v["frac_of_peak"] = v["tflops"] / p if p else None
+            if not (dims.quant and nm != "attention"):
+                v["frac_of_sustained"] = v["tflops"] / peaks["bf16_tflops_sustained"]
         if nm in bt and v["ms"] > 0:
             v["gbs"] = bt[nm] / (v["ms"] / 1e3) / 1e9
             v["frac_of_peak"] = v["gbs"] / peaks["hbm_gbs"]
@@ -295,16 +330,18 @@ def run_gpu_case(torch, j, hi, name, steps, warmup, device, peaks, int8_peak, cl
     if dominant in fl:
         quant_gemm = dims.quant and dominant != "attention"
         roof = {"kernel": dominant, "bound": "tensor", "achieved": d["tflops"],
-                "peak": int8_peak if quant_gemm else tens_peak, "unit": "TOPS" if quant_gemm else "TFLOP/s",
-                "peak_kind": ("int8 torch._int_mm 8192^3 burst, measured in this run" if quant_gemm
-                              else f"bf16 sustained ({peaks['source']})")}
+                "peak": i8_peak if quant_gemm else tens_peak, "unit": "TOPS" if quant_gemm else "TFLOP/s",
+                "peak_kind": (int8_peak["source"] if quant_gemm else f"bf16 burst, of {peaks['source']}")}
     else:
         roof = {"kernel": dominant, "bound": "hbm", "achieved": d["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "peak_kind": f"hbm copy ({peaks['source']})"}
+                "peak_kind": f"hbm copy, of {peaks['source']}"}
     roof["frac"] = roof["achieved"] / roof["peak"] if roof["peak"] else None
     roof["traffic"] = recorded_traffic(dominant, name)
+    ideal_s = sum(fl[k] / ((i8_peak if (dims.quant and k != "attention") else tens_peak) * 1e12)
+                  for k in fl) + sum(bt.values()) / (peaks["hbm_gbs"] * 1e9)
     res = {"workload": name, "n_rows": n, "n_valid": lay.n_valid, "n_pad": lay.n_pad,
            "seconds": secs_max, "ms_per_step": secs_max / steps * 1e3,
+           "block_frac_of_ideal": ideal_s / (secs_max / steps),
            "value": aggregate_throughput(n, steps, int(os.environ.get("WORLD_SIZE", "1")), secs_max),
            "kernels": kernels, "roofline": roof, "clocks": clk,
            "gpu_launches": steps * ((10 if dims.quant else 8) + (2 if density < 1.0 else 0))}
@@ -324,6 +361,12 @@ def run_gpu_case(torch, j, hi, name, steps, warmup, device, peaks, int8_peak, cl
     del ws, w, out, x
     torch.cuda.empty_cache()
     return res
+
+
+def compact_kernels(kernels):
+    """{interval: [ms, fraction of its roofline]} with 4 significant digits."""
+    return {k: [float(f"{v['ms']:.4g}"), (float(f"{v['frac_of_peak']:.3g}") if v.get("frac_of_peak") else None)]
+            for k, v in kernels.items() if k != "prep"}
 
 
 def run_e2e(torch, blk, inp, w, ws, steps, warmup, device):
@@ -506,6 +549,24 @@ def cpu_oracle_sample(name="t2va_32k", kv_rows=1024, q_rows=8, seed=0):
 
 # --------------------------------------------------------------------------- main
 
+def headline_config(hi, workload, world):
+    """The `config` object of the JSON line; both arms print the same one."""
+    dims, lay = hi.workload(workload)
+    return {"workload": workload, "n_rows": lay.n, "n_valid": lay.n_valid, "hidden": dims.hidden,
+            "heads": dims.heads, "head_dim": dims.head_dim, "ffn": dims.ffn, "parallelism": f"replicas x{world}",
+            "flush": "none: inputs (352 MB) and weights (771 MB) exceed the 126 MB L2"}
+
+
+def r4(v):
+    return float(f"{v:.4g}") if isinstance(v, (int, float)) and v is not None else v
+
+
+def extra(name, obj):
+    """Secondary results, one plain-text line each, printed before the JSON
+    line so that the JSON line is the last line of the output."""
+    print(f"extra {name}: " + json.dumps(obj), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -516,11 +577,13 @@ def main():
     ap.add_argument("--no-w8a8", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip real_8k, the padded 32k and ref2va_54k legs")
     ap.add_argument("--no-model", action="store_true", help="skip the whole-model forward legs")
     ap.add_argument("--no-sparse", action="store_true", help="skip the block-sparse attention leg")
     args = ap.parse_args()
     assert args.warmup >= 3 or args.impl == "reference", "at least 3 warm-up steps"
     ws_, rank, local = dist_env()
+    import h3_inputs as hi
 
     if args.impl == "reference":
         if rank != 0:
@@ -536,7 +599,7 @@ def main():
         line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.mean(per_step) * 1e3,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-                "data": "synthetic", "config": {"workload": args.workload, "n_rows": 32768, "flush": "none (CPU)"},
+                "data": "synthetic", "config": headline_config(hi, args.workload, ws_),
                 "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc},
                 "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
@@ -547,53 +610,84 @@ def main():
     world, rank = init_dist(backend)
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
-    import h3_inputs as hi
     import joint_video_audio_b200 as j
     peaks = load_peaks()
     int8_peak = measure_int8_peak(torch, device)
-    clocks = ClockSampler(local)
+    cache = WeightCache(torch, j, hi, device)
     main_res = run_gpu_case(torch, j, hi, args.workload, args.steps, args.warmup, device, peaks, int8_peak,
-                            clocks=clocks, e2e=not args.no_e2e)
+                            clocks=ClockSampler(local), e2e=not args.no_e2e, cache=cache)
     w8 = None
     if not args.no_w8a8:
-        w8 = run_gpu_case(torch, j, hi, "w8a8_t2va_32k", args.steps, args.warmup, device, peaks, int8_peak)
-    modt = run_modulation(torch, j, hi, device, peaks, args.steps)
+        w8 = run_gpu_case(torch, j, hi, "w8a8_t2va_32k", args.steps, args.warmup, device, peaks, int8_peak,
+                          clocks=ClockSampler(local), e2e=not args.no_e2e, cache=cache)
+    others = {}
+    if not args.no_configs:
+        for name in ("real_8k", "t2va_32k_pad168", "ref2va_54k"):
+            others[name] = run_gpu_case(torch, j, hi, name, args.steps, args.warmup, device, peaks, int8_peak,
+                                        clocks=ClockSampler(local), cache=cache)
     sparse = None
     if not args.no_sparse:
         sp = run_gpu_case(torch, j, hi, args.workload, args.steps, args.warmup, device, peaks, int8_peak,
-                          density=0.25)
+                          density=0.25, cache=cache)
         sparse = {"workload": sp["workload"], "value": sp["value"], "unit": UNIT, "ms_per_step": sp["ms_per_step"],
                   **sp["sparse"], "gpu_launches": sp["gpu_launches"]}
+    del cache
+    torch.cuda.empty_cache()
+    modt = run_modulation(torch, j, hi, device, peaks, args.steps)
     models = []
     if not args.no_model:
         for q in (0, 1):
             models.append(run_model(torch, j, hi, device, min(args.steps, 3), 3, q))
-    cpu = None
+    cpu = cpu8 = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rps, secs, desc, threads = cpu_oracle_sample(args.workload)
         cpu = {"value": rps, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc,
                "sample_seconds": secs}
+        if w8:
+            rps, secs, desc, threads = cpu_oracle_sample("w8a8_t2va_32k")
+            cpu8 = {"value": rps, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc,
+                    "sample_seconds": secs}
     if rank == 0:
-        roof = dict(main_res["roofline"])
+        # full detail first, as plain-text lines
+        extra("bf16_kernels", main_res["kernels"])
+        if w8:
+            extra("w8a8", {k: w8[k] for k in ("workload", "value", "ms_per_step", "roofline", "kernels", "clocks",
+                                               "e2e", "gpu_launches", "block_frac_of_ideal")} | {"cpu_baseline": cpu8})
+        for name, r in others.items():
+            extra(name, {k: r[k] for k in ("n_rows", "n_valid", "n_pad", "value", "ms_per_step", "roofline",
+                                           "kernels", "clocks", "gpu_launches", "block_frac_of_ideal")})
+        if sparse:
+            extra("sparse_attention", sparse)
+        extra("modulation_table", modt)
+        for m in models:
+            extra(f"model_forward_{m['mode']}", m)
+        extra("peaks", {"bf16_burst_tflops": peaks["bf16_tflops"], "bf16_sustained_tflops": peaks["bf16_tflops_sustained"],
+                        "hbm_gbs": peaks["hbm_gbs"], "source": peaks["source"], "int8": int8_peak})
+        # the JSON line: compact, so that it fits whole in a short log tail
+        roof = {k: r4(v) for k, v in main_res["roofline"].items()}
         line = {"metric": METRIC, "value": main_res["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": main_res["ms_per_step"], "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": {"workload": args.workload, "n_rows": main_res["n_rows"], "n_valid": main_res["n_valid"],
-                           "hidden": 5376, "heads": 56, "head_dim": 128, "ffn": 14336,
-                           "parallelism": f"replicas x{world}",
-                           "flush": "none: inputs (352 MB) and weights (771 MB) exceed the 126 MB L2"},
+                "config": headline_config(hi, args.workload, world),
                 "roofline": roof, "cpu_baseline": cpu, "e2e": main_res.get("e2e"),
                 "gpu_launches": main_res["gpu_launches"], "clocks": main_res["clocks"],
-                "kernels": main_res["kernels"], "int8_peak_tops": int8_peak}
+                "block_frac_of_ideal": r4(main_res["block_frac_of_ideal"]),
+                "kernels_ms_frac": compact_kernels(main_res["kernels"])}
         if w8:
-            line["w8a8"] = {"workload": w8["workload"], "value": w8["value"], "unit": UNIT,
-                            "ms_per_step": w8["ms_per_step"], "roofline": w8["roofline"], "kernels": w8["kernels"],
-                            "gpu_launches": w8["gpu_launches"]}
-        line["modulation_table"] = modt
-        if models:
-            line["model_forward"] = models
-        if sparse:
-            line["sparse_attention"] = sparse
+            line["w8a8"] = {"workload": w8["workload"], "value": r4(w8["value"]), "ms_per_step": r4(w8["ms_per_step"]),
+                            "e2e_value": r4(w8["e2e"]["value"]) if w8.get("e2e") else None,
+                            "block_frac_of_ideal": r4(w8["block_frac_of_ideal"]),
+                            "roofline": {k: r4(v) for k, v in w8["roofline"].items() if k != "peak_kind"},
+                            "clocks_sm_mhz": (w8["clocks"] or {}).get("sm_mhz"),
+                            "clocks_reasons": (w8["clocks"] or {}).get("reasons"),
+                            "cpu_baseline_value": r4(cpu8["value"]) if cpu8 else None,
+                            "kernels_ms_frac": compact_kernels(w8["kernels"])}
+        if others:
+            line["configs"] = {name: {"value": r4(r["value"]), "ms_per_step": r4(r["ms_per_step"]),
+                                      "attention_frac": r4(r["kernels"]["attention"].get("frac_of_peak")),
+                                      "block_frac_of_ideal": r4(r["block_frac_of_ideal"])}
+                               for name, r in others.items()}
+        line["int8_peak_tops"] = r4(int8_peak["tops"]) if int8_peak else None
         print(json.dumps(line), flush=True)
     import torch.distributed as dist
     if dist.is_initialized():

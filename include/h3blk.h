@@ -207,6 +207,19 @@ H3BLK_API int h3blk_set_attention_density(h3blk_handle h, float density);
 #define H3BLK_TIMING_POINTS 11
 H3BLK_API int h3blk_set_kernel_events(h3blk_handle h, void* const* events, int n_events);
 
+/* Test-only, W8A8 handles: when gemm is 0 (QKV), 1 (out-projection), 2 (FFN
+ * up, W1 | W3) or 3 (FFN down), every later h3blk_forward on this handle also
+ * writes that int8 GEMM's raw int32 accumulators, as its epilogue reads them
+ * from tensor memory before dequantisation, to `buf` as int32
+ * [n_rows, weight rows] row-major (weight rows: 3*heads*head_dim, hidden,
+ * 2*ffn, hidden). The integer product of the rotated W8A8 linears ("HyperFlow
+ * H3 Flash ...", "How it got smaller and faster") can then be checked bit for
+ * bit against the GPU's own int8 operands. `buf` is caller-owned device
+ * memory (16-byte aligned) of `bytes`; a forward whose rows need more returns
+ * INVALID_ARG before launching the GEMM. gemm = -1 switches it off.
+ * UNSUPPORTED on a bf16 handle; INVALID_ARG for other values. */
+H3BLK_API int h3blk_set_debug_accumulators(h3blk_handle h, int gemm, void* buf, size_t bytes);
+
 /* --------------------------------------------------------------- W8A8 */
 /* Bytes of the int8 weight blob for this configuration. */
 H3BLK_API int h3blk_int8_weights_bytes(h3blk_handle h, size_t* bytes);
@@ -427,14 +440,28 @@ H3BLK_API int h3blk_ulysses_out(h3blk_handle h, int64_t n_rows, const h3blk_ulys
  *   qkv  bf16 [N, 3*heads*head_dim]  (the layout of H3BLK_STAGE_QKV)
  *   tag, tidx int32 [N]              (as for h3blk_forward; tidx only validated)
  *   o    bf16 [N, heads*head_dim]    output
- * UNSUPPORTED when n_rows > 524,288 (the fixed scratch's limit) or head_dim is
- * not 64 / 128. It calls no allocator. All calls share the one scratch array,
- * which keeps the last call's contents: calls that overlap on the GPU race,
- * so serialise them. The first call on each device looks up the array's
- * device address; make that first call before any stream capture. */
+ * UNSUPPORTED when n_rows > 524,288 (the fixed scratch's limit), head_dim is
+ * not 64 / 128, or heads*head_dim > 16384. It calls no allocator. All calls
+ * share the one scratch array, which keeps the last call's contents: calls
+ * that overlap on the GPU race, so serialise them. The first call on each
+ * device looks up the array's device address and keeps it for the life of
+ * the process (it assumes the device's primary context is never reset); make
+ * that first call before any stream capture. Errors the kernels find (a tag
+ * or timestep index outside the table, a pipeline wait that ran out) are not
+ * in the return value, which only covers the launch: read them with
+ * h3blk_attention_noalloc_check. */
 H3BLK_API int h3blk_attention_noalloc(int64_t n_rows, int heads, int head_dim, int n_tags, int n_t,
                                       const void* qkv, const int32_t* tag, const int32_t* tidx, void* o,
                                       void* stream);
+
+/* Status of the last h3blk_attention_noalloc call on the current device:
+ * synchronises `stream`, reads the error word of the fixed scratch array (a
+ * copy into host memory, no allocation) and sets *status to H3BLK_OK,
+ * H3BLK_ERR_BAD_INDEX (a tag or timestep index outside the table) or
+ * H3BLK_ERR_TIMEOUT (a pipeline wait ran out; the output is incomplete).
+ * Every call resets the word, so the status covers the latest call only.
+ * INVALID_ARG for a null status. The pages have no counterpart either. */
+H3BLK_API int h3blk_attention_noalloc_check(void* stream, int* status);
 
 /* Test-only: runs, on `stream`, one bounded wait of the kind every pipeline
  * wait of this library is (an mbarrier phase polled against a time limit), on
@@ -446,6 +473,16 @@ H3BLK_API int h3blk_attention_noalloc(int64_t n_rows, int heads, int head_dim, i
  * caller-owned device int32 (4-byte aligned) used as the error word; it is
  * reset by the call. INVALID_ARG for a null pointer or a limit out of range. */
 H3BLK_API int h3blk_selftest_wait(int complete, int limit_ms, void* word, void* stream, int* status);
+
+/* Test-only: y[i] = the polynomial 2^x[i] that the attention kernel
+ * evaluates on the FMA pipe for a share of its softmax exponentials (2^n by
+ * exponent-field addition times a degree-3 fit of 2^f on [-1/2, 1/2]; inputs
+ * below -125 are clamped to -125). x and y are caller-owned device fp32 [n],
+ * asynchronous on `stream`. Stated error: relative <= 1e-4 for x in
+ * [-125, 8]. INVALID_ARG for null pointers or n outside [1, 2^30]. The
+ * softmax of "MiniMaxH3Transformer3DModel" (full self-attention) is where it
+ * is used. */
+H3BLK_API int h3blk_selftest_exp2(const float* x, float* y, int64_t n, void* stream);
 
 /* Message for a status code (static storage). */
 H3BLK_API const char* h3blk_error_string(int status);

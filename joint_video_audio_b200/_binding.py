@@ -27,12 +27,13 @@ STAGE = {name: i for i, name in enumerate(STAGES)}
 EXPORTS = ["h3blk_create", "h3blk_destroy", "h3blk_workspace_bytes", "h3blk_stage_view", "h3blk_forward",
            "h3blk_check", "h3blk_int8_weights_bytes", "h3blk_prepare_int8_weights", "h3blk_rotate_quantize",
            "h3blk_gemm_s8_s32", "h3blk_gemm_bf16", "h3blk_error_string", "h3blk_version",
-           "h3blk_set_kernel_events", "h3blk_attention_noalloc", "h3blk_modulation_scratch_bytes",
+           "h3blk_set_kernel_events", "h3blk_attention_noalloc", "h3blk_attention_noalloc_check",
+           "h3blk_modulation_scratch_bytes",
            "h3blk_modulation_table", "h3blk_model_workspace_bytes", "h3blk_model_forward", "h3blk_model_check",
            "h3blk_model_graph_create", "h3blk_graph_launch", "h3blk_graph_info", "h3blk_graph_destroy",
            "h3blk_ulysses_buffer_bytes", "h3blk_ulysses_workspace_bytes", "h3blk_ulysses_qkv",
            "h3blk_ulysses_attention", "h3blk_ulysses_out", "h3blk_set_attention_density",
-           "h3blk_selftest_wait"]
+           "h3blk_selftest_wait", "h3blk_selftest_exp2", "h3blk_set_debug_accumulators"]
 
 H3BLK_MAX_RANKS = 8
 
@@ -120,7 +121,10 @@ def _load():
         "h3blk_version": (i32, []),
         "h3blk_set_kernel_events": (i32, [vp, C.POINTER(vp), i32]),
         "h3blk_attention_noalloc": (i32, [i64, i32, i32, i32, i32, vp, vp, vp, vp, vp]),
+        "h3blk_attention_noalloc_check": (i32, [vp, C.POINTER(i32)]),
         "h3blk_selftest_wait": (i32, [i32, i32, vp, vp, C.POINTER(i32)]),
+        "h3blk_selftest_exp2": (i32, [vp, vp, i64, vp]),
+        "h3blk_set_debug_accumulators": (i32, [vp, i32, vp, C.c_size_t]),
         "h3blk_modulation_scratch_bytes": (i32, [vp, C.POINTER(h3blk_mod_weights), C.POINTER(sz)]),
         "h3blk_modulation_table": (i32, [vp, C.POINTER(h3blk_mod_weights), C.POINTER(C.c_float),
                                           C.POINTER(C.c_float), C.c_float, vp, vp, sz, vp]),
@@ -257,6 +261,15 @@ def h3blk_attention_noalloc(n_rows, heads, head_dim, n_tags, n_t, qkv, tag, tidx
     return _lib.h3blk_attention_noalloc(n_rows, heads, head_dim, n_tags, n_t, qkv, tag, tidx, o, stream)
 
 
+def h3blk_attention_noalloc_check(stream) -> int:
+    """Synchronises `stream` and returns the device-side status of the last
+    h3blk_attention_noalloc call (H3BLK_OK, H3BLK_ERR_BAD_INDEX or
+    H3BLK_ERR_TIMEOUT)."""
+    st = C.c_int32()
+    _check("h3blk_attention_noalloc_check", _lib.h3blk_attention_noalloc_check(stream, C.byref(st)))
+    return st.value
+
+
 def h3blk_selftest_wait(complete: bool, limit_ms: int, word, stream) -> int:
     """Test-only: one bounded pipeline wait on a barrier that completes
     (complete=True) or never does; returns the status h3blk_check would give
@@ -264,6 +277,18 @@ def h3blk_selftest_wait(complete: bool, limit_ms: int, word, stream) -> int:
     st = C.c_int32()
     _check("h3blk_selftest_wait", _lib.h3blk_selftest_wait(1 if complete else 0, limit_ms, word, stream, C.byref(st)))
     return st.value
+
+
+def h3blk_set_debug_accumulators(handle, gemm: int, buf, nbytes: int) -> None:
+    """Test-only (W8A8): later forwards also dump int8 GEMM `gemm`'s raw int32
+    accumulators (0 QKV, 1 out-proj, 2 FFN up, 3 FFN down; -1 off) to `buf`."""
+    _check("h3blk_set_debug_accumulators", _lib.h3blk_set_debug_accumulators(handle, gemm, buf, nbytes))
+
+
+def h3blk_selftest_exp2(x, y, n, stream) -> None:
+    """Test-only: y = the attention's FMA-pipe polynomial 2^x (device fp32
+    pointers, n elements)."""
+    _check("h3blk_selftest_exp2", _lib.h3blk_selftest_exp2(x, y, n, stream))
 
 
 def h3blk_modulation_scratch_bytes(handle, w: h3blk_mod_weights) -> int:

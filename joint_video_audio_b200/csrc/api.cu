@@ -197,6 +197,17 @@ size_t block_workspace_bytes(const h3blk_config& c, int64_t n, int keep_per_1024
   } while (0)
 
 namespace {
+// Test-only: routes the s32 accumulators of int8 GEMM `which` (0 QKV, 1
+// out-projection, 2 FFN up, 3 FFN down) to the caller's buffer when that dump
+// is switched on; INVALID_ARG if the buffer cannot hold [M, Nb] int32.
+int attach_dump(const h3blk_ctx* h, int which, GemmArgs& g) {
+  if (h->dbg_gemm != which || !g.int8) return H3BLK_OK;
+  if ((size_t)g.M * (size_t)g.Nb * sizeof(int32_t) > h->dbg_bytes) return H3BLK_ERR_INVALID_ARG;
+  g.acc_dump = h->dbg_buf;
+  g.ld_dump = g.Nb;
+  return H3BLK_OK;
+}
+
 cudaError_t mark(const h3blk_ctx* h, bool timing, int i, cudaStream_t s) {
   return timing ? cudaEventRecord(h->events[i], s) : cudaSuccess;
 }
@@ -258,6 +269,7 @@ int phase_qkv(const h3blk_ctx* h, const Span& sp, const void* x, const int32_t* 
     g.route_row0 = sp.row0;
     for (int r = 0; r < route->ranks; ++r) g.route_dst[r] = route->dst[r];
   }
+  if (int st = attach_dump(h, 0, g)) return st;
   H3_TRY(mark(h, timing, 2, s));
   H3_TRY(h3::launch_gemm(g, enc, sms, s));
   return H3BLK_OK;
@@ -337,6 +349,7 @@ int phase_out(const h3blk_ctx* h, const Span& sp, const void* x, const int32_t* 
   g.gate_idx = 2;
   g.s_a = q ? b.o_s : nullptr;
   g.s_b = w->s_o;
+  if (int st = attach_dump(h, 1, g)) return st;
   H3_TRY(mark(h, timing, 5, s));
   H3_TRY(h3::launch_gemm(g, enc, sms, s));
   H3_TRY(mark(h, timing, 6, s));
@@ -374,6 +387,7 @@ int phase_out(const h3blk_ctx* h, const Span& sp, const void* x, const int32_t* 
   g.ld_out = F;
   g.s_a = q ? b.h2_s : nullptr;
   g.s_b = w->s_13;
+  if (int st = attach_dump(h, 2, g)) return st;
   H3_TRY(mark(h, timing, 7, s));
   H3_TRY(h3::launch_gemm(g, enc, sms, s));
   H3_TRY(mark(h, timing, 8, s));
@@ -397,6 +411,7 @@ int phase_out(const h3blk_ctx* h, const Span& sp, const void* x, const int32_t* 
   g.gate_idx = 5;
   g.s_a = q ? b.a_s : nullptr;
   g.s_b = w->s_2;
+  if (int st = attach_dump(h, 3, g)) return st;
   H3_TRY(mark(h, timing, 9, s));
   H3_TRY(h3::launch_gemm(g, enc, sms, s));
   H3_TRY(mark(h, timing, 10, s));
@@ -484,6 +499,9 @@ int h3blk_create(const h3blk_config* cfg, h3blk_handle* out) {
   h->cfg = c;
   h->timing = false;
   h->keep_per_1024 = 1024;
+  h->dbg_gemm = -1;
+  h->dbg_buf = nullptr;
+  h->dbg_bytes = 0;
   for (auto& e : h->events) e = nullptr;
   const int pairs[3] = {c.rope_pairs_t, c.rope_pairs_h, c.rope_pairs_w};
   int j = 0;
@@ -514,6 +532,22 @@ int h3blk_set_kernel_events(h3blk_handle h, void* const* events, int n_events) {
     h->events[i] = reinterpret_cast<cudaEvent_t>(events[i]);
   }
   h->timing = true;
+  return H3BLK_OK;
+}
+
+int h3blk_set_debug_accumulators(h3blk_handle h, int gemm, void* buf, size_t bytes) {
+  if (!h || gemm < -1 || gemm > 3) return H3BLK_ERR_INVALID_ARG;
+  if (gemm == -1) {
+    h->dbg_gemm = -1;
+    h->dbg_buf = nullptr;
+    h->dbg_bytes = 0;
+    return H3BLK_OK;
+  }
+  if (h->cfg.quant == 0) return H3BLK_ERR_UNSUPPORTED;
+  if (!buf || !aligned16(buf) || bytes == 0) return H3BLK_ERR_INVALID_ARG;
+  h->dbg_gemm = gemm;
+  h->dbg_buf = static_cast<int32_t*>(buf);
+  h->dbg_bytes = bytes;
   return H3BLK_OK;
 }
 

@@ -13,6 +13,10 @@ struct h3blk_ctx {
   cudaEvent_t events[H3BLK_TIMING_POINTS];
   bool timing;
   int keep_per_1024;  // 1024: dense attention; below: block-sparse
+  // test-only dump of one int8 GEMM's s32 accumulators (-1: off)
+  int dbg_gemm;
+  int32_t* dbg_buf;
+  size_t dbg_bytes;
 };
 
 namespace h3api {

@@ -115,9 +115,15 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&
 }
 
 template <bool INT8>
-__device__ __forceinline__ void load_chunk(uint32_t taddr, float sa, const float* sb, int col, float (&v)[32]) {
+__device__ __forceinline__ void load_chunk(uint32_t taddr, float sa, const float* sb, int col, float (&v)[32],
+                                           int32_t* dump = nullptr) {
   uint32_t r[32];
   tmem_ld32(taddr, r);
+  if (INT8 && dump) {
+    uint4* d = reinterpret_cast<uint4*>(dump + col);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) d[i] = make_uint4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
+  }
 #pragma unroll
   for (int j = 0; j < 32; ++j) v[j] = acc_value<INT8>(r[j], sa, sb, col + j);
 }
@@ -143,13 +149,14 @@ template <int EPI, bool INT8>
 __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tacc, int64_t row, bool row_ok, int n_tile,
                                               int half) {
   const float sa = (INT8 && row_ok) ? __ldg(p.s_a + row) : 0.f;
+  int32_t* dump = (INT8 && p.acc_dump && row_ok) ? p.acc_dump + row * p.ld_dump : nullptr;
   if (EPI == kEpiSwiGLU) {
     const int col0 = n_tile * 128;
 #pragma unroll 1
     for (int c = 2 * half; c < 2 * half + 2; ++c) {
       float g[32], u[32];
-      load_chunk<INT8>(tacc + c * 32, sa, p.s_b, col0 + c * 32, g);
-      load_chunk<INT8>(tacc + 128 + c * 32, sa, p.s_b, p.N + col0 + c * 32, u);
+      load_chunk<INT8>(tacc + c * 32, sa, p.s_b, col0 + c * 32, g, dump);
+      load_chunk<INT8>(tacc + 128 + c * 32, sa, p.s_b, p.N + col0 + c * 32, u, dump);
 #pragma unroll
       for (int j = 0; j < 32; ++j) g[j] = g[j] / (1.f + __expf(-g[j])) * u[j];
       if (row_ok) store_bf16x32(reinterpret_cast<__nv_bfloat16*>(p.out) + row * p.ld_out + col0 + c * 32, g);
@@ -184,7 +191,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tacc, 
       const int col = n0 + c * 32;
       if (col >= p.N) break;
       float v[32];
-      load_chunk<INT8>(tacc + c * 32, sa, p.s_b, col, v);
+      load_chunk<INT8>(tacc + c * 32, sa, p.s_b, col, v, dump);
       if (!row_ok) continue;
       __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + row * p.ld_out + col;
       if (EPI == kEpiStoreBf16 && p.bias) {
@@ -252,7 +259,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tacc, 
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           float v[32];
-          load_chunk<INT8>(th + c * 32, sa, p.s_b, col0 + c * 32, v);
+          load_chunk<INT8>(th + c * 32, sa, p.s_b, col0 + c * 32, v, dump);
           if (row_ok) store_bf16x32(dst + c * 32, v);
         }
         continue;
@@ -261,7 +268,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tacc, 
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         float v[32];
-        load_chunk<INT8>(th + c * 32, sa, p.s_b, col0 + c * 32, v);
+        load_chunk<INT8>(th + c * 32, sa, p.s_b, col0 + c * 32, v, dump);
 #pragma unroll
         for (int j = 0; j < 32; ++j) ss = fmaf(v[j], v[j], ss);
       }
@@ -270,7 +277,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tacc, 
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         float v[32];
-        load_chunk<INT8>(th + c * 32, sa, p.s_b, col0 + c * 32, v);
+        load_chunk<INT8>(th + c * 32, sa, p.s_b, col0 + c * 32, v, dump);
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = v[j] * rstd * __bfloat162float(gain[c * 32 + j]);
 #pragma unroll

@@ -104,6 +104,11 @@ struct GemmArgs {
   int route_ranks = 0, route_hg = 0;
   int64_t route_row0 = 0;
   void* route_dst[kMaxRanks] = {};
+  // int8 mode, test-only: when set, the epilogue also writes every raw s32
+  // accumulator it reads to acc_dump[row * ld_dump + b_row] (b_row = the
+  // weight row the value belongs to)
+  int32_t* acc_dump = nullptr;
+  int64_t ld_dump = 0;
 };
 cudaError_t launch_gemm(const GemmArgs& a, PFN_cuTensorMapEncodeTiled_v12000 encode, int num_sms, cudaStream_t s);
 

@@ -20,7 +20,14 @@
 //     on the same device) race with each other; serialise them;
 //   * the first call on each device looks up the array's device address
 //     (cudaGetSymbolAddress, with that device current) and caches it; make that
-//     first call before any stream capture.
+//     first call before any stream capture. The cached address assumes the
+//     device's primary context lives as long as the process: after a
+//     cudaDeviceReset the cache is stale, and the library must not be called
+//     again in that process;
+//   * errors found on the device (an out-of-range tag or timestep index, a
+//     pipeline wait that ran out) go to an error word inside the array;
+//     h3blk_attention_noalloc_check reads it, so call it after each call (or
+//     each batch of calls) whose output must be trusted.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -29,6 +36,7 @@
 
 #include "../../include/h3blk.h"
 #include "kernels.cuh"
+#include "ptx.cuh"
 
 namespace {
 
@@ -36,6 +44,7 @@ constexpr int64_t kNoAllocMaxTiles = 4096;                 // 128-row tiles
 constexpr int64_t kNoAllocMaxRows = kNoAllocMaxTiles * 128;  // 524,288 rows
 constexpr size_t kNoAllocErrorBytes = 256;                 // error word, padded
 constexpr size_t kNoAllocScratchBytes = kNoAllocErrorBytes + kNoAllocMaxTiles * sizeof(h3::TileInfo);
+constexpr int kNoAllocMaxHeadChannels = 16384;             // heads * head_dim, as h3blk_create allows
 
 // The scratch itself. In host code this name only stands for the array: its
 // device address comes from cudaGetSymbolAddress below.
@@ -85,6 +94,7 @@ extern "C" int h3blk_attention_noalloc(int64_t n_rows, int heads, int head_dim, 
   if (n_rows < 1 || heads < 1 || n_tags < 1 || n_t < 1 || !qkv || !tag || !tidx || !o) return H3BLK_ERR_INVALID_ARG;
   if (!aligned16(qkv) || !aligned16(o) || !aligned16(tag) || !aligned16(tidx)) return H3BLK_ERR_INVALID_ARG;
   if (head_dim != 64 && head_dim != 128) return H3BLK_ERR_UNSUPPORTED;
+  if (heads > kNoAllocMaxHeadChannels / head_dim) return H3BLK_ERR_UNSUPPORTED;  // the block's own limit
   if (n_rows > kNoAllocMaxRows) return H3BLK_ERR_UNSUPPORTED;  // beyond the fixed scratch
   void* scratch = nullptr;
   PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
@@ -106,4 +116,23 @@ extern "C" int h3blk_attention_noalloc(int64_t n_rows, int heads, int head_dim, 
   a.head_dim = head_dim;
   a.err = err;
   return h3::launch_attention(a, enc, s) == cudaSuccess ? H3BLK_OK : H3BLK_ERR_CUDA;
+}
+
+extern "C" int h3blk_attention_noalloc_check(void* stream, int* status) {
+  if (!status) return H3BLK_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return H3BLK_ERR_CUDA;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return H3BLK_ERR_CUDA;
+  int bits = 0;
+  // the error word is the first int of the array; a device on which no call
+  // ran yet reads the array's initial zero
+  if (cudaMemcpyFromSymbol(&bits, g_noalloc_scratch, sizeof(int), 0, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return H3BLK_ERR_CUDA;
+  if (bits & (h3::kErrTimeoutGemm | h3::kErrTimeoutAttn | h3::kErrTimeoutStream))
+    *status = H3BLK_ERR_TIMEOUT;
+  else if (bits & (h3::kErrBadIndex | h3::kErrBadRowIndex))
+    *status = H3BLK_ERR_BAD_INDEX;
+  else
+    *status = H3BLK_OK;
+  return H3BLK_OK;
 }

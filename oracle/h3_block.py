@@ -310,8 +310,9 @@ class BlockOracle:
         quantises them straight from fp32)."""
         return bf16_round(a) if (self.faithful and not self.quant) else a
 
-    # linear y = a W^T, bf16 weights or rotated W8A8; ``rows`` selects output
-    # channels (weight rows), which leaves every computed column unchanged
+    # linear y = a W^T, bf16 weights or rotated W8A8; ``rows`` (a slice)
+    # selects output channels (weight rows), which leaves every computed
+    # column unchanged
     def linear(self, a, name, rows=None):
         if self.quant:
             wq, sw = self.int8[name]
@@ -332,9 +333,9 @@ class BlockOracle:
         d = self.d
         HD = d.hd
         names = [p for p in ("q", "k", "v") if p in part]
-        idx = {"q": 0, "k": 1, "v": 2}
-        cols = np.concatenate([np.arange(idx[p] * HD, (idx[p] + 1) * HD) for p in names])
-        y = self.linear(h1, "qkv", rows=None if len(names) == 3 else cols)
+        first = {"q": 0, "k": 1, "v": 2}[names[0]]
+        assert [{"q": 0, "k": 1, "v": 2}[p] for p in names] == list(range(first, first + len(names)))
+        y = self.linear(h1, "qkv", rows=slice(first * HD, (first + len(names)) * HD))
         ys = {p: y[:, i * HD:(i + 1) * HD] for i, p in enumerate(names)}
         out = {}
         if "q" in part:

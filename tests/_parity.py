@@ -96,3 +96,10 @@ def rows_of(t, rows):
     if rows is None:
         return t
     return t[torch.as_tensor(rows, device=t.device)]
+
+
+def blob_tensor(dw, ptr, numel, dtype):
+    """View of one array inside the int8 weight blob written by the library."""
+    off = ptr - dw.blob.data_ptr()
+    nbytes = numel * torch.tensor([], dtype=dtype).element_size()
+    return dw.blob[off:off + nbytes].view(dtype)

@@ -388,3 +388,33 @@ def test_block_sparse_mode_sizes_block_and_model_workspaces():
     blk.set_attention_density(1.0)
     assert blk.workspace_bytes(320) == dense_blk
     assert B.h3blk_model_workspace_bytes(blk.handle, mc, w.time, 320, 64) == dense_model
+
+
+def test_debug_accumulator_dump_validation():
+    """The test-only s32 accumulator dump: W8A8 handles only, gemm in -1..3,
+    a non-null 16-byte aligned buffer; -1 switches it off."""
+    from dataclasses import replace
+    lib = B._lib
+    bf = j.H3Block(hi.TINY)
+    assert lib.h3blk_set_debug_accumulators(bf.handle, 0, 1 << 20, 4096) == B.H3BLK_ERR_UNSUPPORTED
+    assert lib.h3blk_set_debug_accumulators(bf.handle, -1, None, 0) == B.H3BLK_OK
+    q = j.H3Block(replace(hi.TINY, quant=1))
+    for gemm in (-2, 4):
+        assert lib.h3blk_set_debug_accumulators(q.handle, gemm, 1 << 20, 4096) == B.H3BLK_ERR_INVALID_ARG
+    assert lib.h3blk_set_debug_accumulators(q.handle, 0, None, 4096) == B.H3BLK_ERR_INVALID_ARG
+    assert lib.h3blk_set_debug_accumulators(q.handle, 0, (1 << 20) + 4, 4096) == B.H3BLK_ERR_INVALID_ARG
+    assert lib.h3blk_set_debug_accumulators(q.handle, 0, 1 << 20, 0) == B.H3BLK_ERR_INVALID_ARG
+    for gemm in range(4):
+        assert lib.h3blk_set_debug_accumulators(q.handle, gemm, 1 << 20, 4096) == B.H3BLK_OK
+    assert lib.h3blk_set_debug_accumulators(q.handle, -1, None, 0) == B.H3BLK_OK
+    assert lib.h3blk_set_debug_accumulators(None, -1, None, 0) == B.H3BLK_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("args", [(0, 0, 1, 0), (1 << 20, 0, 4, 0), (0, 1 << 20, 4, 0), (1 << 20, 1 << 21, 0, 0),
+                                  (1 << 20, 1 << 21, (1 << 30) + 1, 0)])
+def test_selftest_exp2_validates_before_gpu(args):
+    assert B._lib.h3blk_selftest_exp2(*args) == B.H3BLK_ERR_INVALID_ARG
+
+
+def test_noalloc_check_validates_status_pointer():
+    assert B._lib.h3blk_attention_noalloc_check(None, None) == B.H3BLK_ERR_INVALID_ARG

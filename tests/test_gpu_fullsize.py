@@ -19,7 +19,7 @@ import torch
 
 import h3_inputs as hi
 from oracle import h3_block as orc
-from tests._parity import GpuCase, assert_intermediate, assert_stage, to64
+from tests._parity import GpuCase, assert_intermediate, assert_stage, blob_tensor, to64
 
 pytestmark = pytest.mark.gpu
 
@@ -156,7 +156,16 @@ def test_end_to_end_vs_oracle(name):
     _check_padding(case)
     rows = hi.sample_rows(lay, k=256, k_pad=8)
     ob = orc.BlockOracle(dims, inp.weights)
-    ref = ob.forward(inp.x, lay.tag, lay.tidx, lay.pos, inp.table, rows=rows)
+    # the oracle's forward in subset mode, its query rows taken 64 at a time
+    # to bound host memory (the attention probabilities of 64 rows over 54k
+    # keys and 56 heads are 1.6 GB in fp64)
+    k_all, v_all = ob.kv_all(inp.x, lay.tag, lay.tidx, lay.pos, inp.table)
+    doc = orc.documents(lay.tag)
+    parts = [ob.query(inp.x[torch.as_tensor(r)], lay.tag[r], lay.tidx[r], lay.pos[r], inp.table, k_all, v_all, doc)
+             for r in np.array_split(rows, max(1, len(rows) // 64))]
+    ref = {key: np.concatenate([p_[key] for p_ in parts]) for key in parts[0]}
+    ref["k"], ref["v"] = k_all[rows], v_all[rows]
+    del k_all, v_all
     if dims.quant:
         # int8 codes of the pre-attention norm (SURVEY reading c24: ties may
         # round either way, so >= 99.9 % identical and never more than 1 apart)
@@ -174,3 +183,40 @@ def test_end_to_end_vs_oracle(name):
     assert_intermediate("x1", _rows_gpu(case.stage("X1"), rows), ref["x1"])
     assert_intermediate("a", _rows_gpu(case.stage("A"), rows), ref["a"])
     assert_stage("out", _rows_gpu(case.out, rows), ref["out"])
+
+
+def test_w8a8_block_accumulators_exact_at_32k():
+    """The int32 accumulators of the block's own four int8 GEMMs (QKV, out-
+    projection, FFN up, FFN down), as their epilogues read them inside
+    h3blk_forward at the W8A8 32k layout, equal bit for bit the exact integer
+    products of the GPU's own int8 operands, on 256 seeded rows and every
+    output column ("HyperFlow H3 Flash ...", "How it got smaller and faster":
+    int8 products, int32 accumulation)."""
+    from joint_video_audio_b200 import _binding as B
+    dims, lay = hi.workload("w8a8_t2va_32k")
+    inp = hi.make_inputs(dims, lay)
+    case = GpuCase(inp)
+    d = dims
+    hd = d.heads * d.head_dim
+    rows = hi.sample_rows(lay, k=256, k_pad=0)
+    ridx = torch.as_tensor(rows, device="cuda")
+    gemms = [  # (index, A operand stage, weight pointer, weight rows, K)
+        (0, "H1_Q8", case.w.c.wqkv, 3 * hd, d.hidden),
+        (1, "O_Q8", case.w.c.wo, d.hidden, hd),
+        (2, "H2_Q8", case.w.c.w13, 2 * d.ffn, d.hidden),
+        (3, "A_Q8", case.w.c.w2, d.hidden, d.ffn),
+    ]
+    try:
+        for which, stage, wptr, nb, K in gemms:
+            buf = torch.zeros((case.n, nb), dtype=torch.int32, device="cuda")
+            B.h3blk_set_debug_accumulators(case.block.handle, which, buf.data_ptr(), buf.numel() * 4)
+            case.run()
+            assert case.block.check(case.ws, case.n) == 0
+            acc = buf[ridx].cpu().numpy().astype(np.int64)
+            a8 = case.stage(stage)[ridx].cpu().numpy()
+            w8 = blob_tensor(case.w, wptr, nb * K, torch.int8).view(nb, K).cpu().numpy()
+            ref = orc.int8_matmul_exact(a8, w8)
+            assert np.array_equal(acc, ref), f"gemm {which}: {int((acc != ref).sum())} accumulators differ"
+            del buf
+    finally:
+        B.h3blk_set_debug_accumulators(case.block.handle, -1, None, 0)

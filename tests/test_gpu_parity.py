@@ -8,7 +8,7 @@ import torch
 
 import h3_inputs as hi
 from oracle import h3_block as orc
-from tests._parity import GpuCase, assert_intermediate, assert_stage, errors, to64
+from tests._parity import GpuCase, assert_intermediate, assert_stage, blob_tensor as _blob_tensor, errors, to64
 
 pytestmark = pytest.mark.gpu
 
@@ -198,13 +198,6 @@ def test_tiny_padding_anywhere():
     ref = orc.BlockOracle(inp.dims, inp.weights).forward(inp.x, lay.tag, lay.tidx, lay.pos, inp.table)
     assert_intermediate("o", case.stage("O"), ref["o"])
     assert_stage("out", case.out, ref["out"])
-
-
-def _blob_tensor(dw, ptr, numel, dtype):
-    """View of one array inside the int8 weight blob written by the library."""
-    off = ptr - dw.blob.data_ptr()
-    nbytes = numel * torch.tensor([], dtype=dtype).element_size()
-    return dw.blob[off:off + nbytes].view(dtype)
 
 
 @pytest.fixture(scope="module")
