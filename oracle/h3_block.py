@@ -169,9 +169,12 @@ def attention(q, k, v, doc_q, doc_k):
         kj = np.nonzero(doc_k == d)[0]
         if kj.size == 0:
             continue
+        # (a document holding every key is used in place: no gathered copy)
+        kd = k if kj.size == k.shape[0] else k[kj]
+        vd = v if kj.size == v.shape[0] else v[kj]
         qh = q[qi].transpose(1, 0, 2)            # [H, rq, D]
-        kh = k[kj].transpose(1, 2, 0)            # [H, D, rk]
-        vh = v[kj].transpose(1, 0, 2)            # [H, rk, D]
+        kh = kd.transpose(1, 2, 0)               # [H, D, rk]
+        vh = vd.transpose(1, 0, 2)               # [H, rk, D]
         p = softmax(np.matmul(qh, kh) / np.sqrt(D))
         out[qi] = np.matmul(p, vh).transpose(1, 0, 2)
     return out
