@@ -651,8 +651,8 @@ def main():
         # full detail first, as plain-text lines
         extra("bf16_kernels", main_res["kernels"])
         if w8:
-            extra("w8a8", {k: w8[k] for k in ("workload", "value", "ms_per_step", "roofline", "kernels", "clocks",
-                                               "e2e", "gpu_launches", "block_frac_of_ideal")} | {"cpu_baseline": cpu8})
+            extra("w8a8", {k: w8.get(k) for k in ("workload", "value", "ms_per_step", "roofline", "kernels", "clocks",
+                                                   "e2e", "gpu_launches", "block_frac_of_ideal")} | {"cpu_baseline": cpu8})
         for name, r in others.items():
             extra(name, {k: r[k] for k in ("n_rows", "n_valid", "n_pad", "value", "ms_per_step", "roofline",
                                            "kernels", "clocks", "gpu_launches", "block_frac_of_ideal")})

@@ -82,6 +82,7 @@ struct Layout {
   size_t off[H3BLK_STAGE_COUNT];
   size_t len[H3BLK_STAGE_COUNT];
   size_t tiles_off;
+  size_t modt_off;
   size_t sp_qsum, sp_ksum, sp_count;  // block-sparse pooling buffers (0 when dense)
   size_t total;
 };
@@ -100,6 +101,8 @@ Layout make_layout(const h3blk_config& c, int64_t n, int keep_per_1024) {
   L.tiles_off = o;
   o = align256(o + ((N + 127) / 128) * sizeof(h3::TileInfo));
   const bool q = c.quant != 0;
+  L.modt_off = o;
+  if (q) o = align256(o + h3::modt_bytes(c.n_tags, c.n_t, c.hidden));
   if (!q) put(H3BLK_STAGE_H1, N * C * 2);
   put(H3BLK_STAGE_QKV, N * 3 * HD * 2);
   put(H3BLK_STAGE_O, N * HD * 2);
@@ -224,6 +227,8 @@ int phase_qkv(const h3blk_ctx* h, const Span& sp, const void* x, const int32_t* 
   if (clear_err) H3_TRY(cudaMemsetAsync(b.err, 0, sizeof(int), s));
   // the tile summary covers the whole sequence: attention reads every row
   H3_TRY(h3::launch_tile_info(tag, tidx, sp.n_total, c.n_tags, c.n_t, b.tiles, b.err, s));
+  // W8A8: the table's pre-norm vectors in the row passes' layout (both pre-norms)
+  if (q) H3_TRY(h3::launch_modt(mod_table, c.n_tags, c.n_t, c.hidden, b.modt, s));
 
   // ---- pre-attention AdaLN + RMSNorm of this call's rows
   h3::ModNormArgs mn;
@@ -238,6 +243,8 @@ int phase_qkv(const h3blk_ctx* h, const Span& sp, const void* x, const int32_t* 
   mn.n_t = c.n_t;
   mn.shift_idx = 0;
   mn.scale_idx = 1;
+  mn.modt = b.modt;
+  mn.modt_v0 = 0;
   mn.eps = c.norm_eps;
   mn.out_q = b.h1_q;
   mn.out_scale = b.h1_s;
@@ -367,6 +374,8 @@ int phase_out(const h3blk_ctx* h, const Span& sp, const void* x, const int32_t* 
   mn.n_t = c.n_t;
   mn.shift_idx = 3;
   mn.scale_idx = 4;
+  mn.modt = b.modt;
+  mn.modt_v0 = 2;
   mn.eps = c.norm_eps;
   mn.out_q = b.h2_q;
   mn.out_scale = b.h2_s;
@@ -427,6 +436,7 @@ int block_forward(const h3blk_ctx* h, int64_t n_rows, const void* x, const int32
   BlockBufs b{};
   b.err = reinterpret_cast<int*>(buf(H3BLK_STAGE_ERROR));
   b.tiles = reinterpret_cast<h3::TileInfo*>(ws + L.tiles_off);
+  b.modt = reinterpret_cast<float4*>(ws + L.modt_off);
   const bool sparse = h->keep_per_1024 < 1024;
   b.sp_qsum = sparse ? reinterpret_cast<float*>(ws + L.sp_qsum) : nullptr;
   b.sp_ksum = sparse ? reinterpret_cast<float*>(ws + L.sp_ksum) : nullptr;

@@ -39,6 +39,7 @@ size_t block_workspace_bytes(const h3blk_config& c, int64_t n, int keep_per_1024
 struct BlockBufs {
   int* err = nullptr;
   h3::TileInfo* tiles = nullptr;
+  float4* modt = nullptr;  // the pre-norm vectors rearranged for the row passes
   // block-sparse selection (null when dense)
   float *sp_qsum = nullptr, *sp_ksum = nullptr;
   int32_t *sp_count = nullptr, *sp_lists = nullptr;

@@ -48,8 +48,17 @@ struct ModNormArgs {
   int8_t* out_q;
   float* out_scale;
   int* err = nullptr;  // device error word (a load that never landed), may be null
+  // the table's shift / (1 + scale) vectors rearranged by launch_modt, and
+  // which pair this pass applies (0: shift1 / scale1, 2: shift2 / scale2)
+  const float4* modt = nullptr;
+  int modt_v0 = 0;
 };
 cudaError_t launch_modnorm(const ModNormArgs& a, cudaStream_t s);
+// Rearranges the table's pre-norm vectors (shift1, 1 + scale1, shift2,
+// 1 + scale2 of every (tag, tidx)) for the row passes: n_tags * n_t * 4 * K
+// floats at `modt`.
+cudaError_t launch_modt(const float* table, int n_tags, int n_t, int K, float4* modt, cudaStream_t s);
+inline size_t modt_bytes(int n_tags, int n_t, int K) { return (size_t)n_tags * n_t * 4 * K * sizeof(float); }
 
 // ---------------------------------------------------------------- K4
 // Rows of a bf16 matrix [rows, K] -> block-128 Hadamard rotation ->

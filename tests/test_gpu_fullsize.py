@@ -19,7 +19,7 @@ import torch
 
 import h3_inputs as hi
 from oracle import h3_block as orc
-from tests._parity import GpuCase, assert_intermediate, assert_stage, blob_tensor, to64
+from tests._parity import GpuCase, assert_intermediate, assert_stage, blob_tensor, errors, to64
 
 pytestmark = pytest.mark.gpu
 
@@ -181,7 +181,17 @@ def test_end_to_end_vs_oracle(name):
     assert_intermediate("v", vg, ref["v"])
     assert_intermediate("o", _rows_gpu(case.stage("O"), rows), ref["o"])
     assert_intermediate("x1", _rows_gpu(case.stage("X1"), rows), ref["x1"])
-    assert_intermediate("a", _rows_gpu(case.stage("A"), rows), ref["a"])
+    if dims.quant:
+        # The FFN-up input is quantised from the GPU's own bf16 x1 on one side
+        # and from the exact x1 on the other: codes near a rounding boundary
+        # differ by one step, so individual SwiGLU outputs differ by int8
+        # quantisation noise, not by bf16 rounding. The stage is held to the
+        # relative RMS bound (the stage chain checks it elementwise from the
+        # GPU's own codes); the block output keeps the full bound below.
+        _, rr = errors(_rows_gpu(case.stage("A"), rows), ref["a"])
+        assert rr <= 1e-2, f"a: rel_rms {rr:.3e}"
+    else:
+        assert_intermediate("a", _rows_gpu(case.stage("A"), rows), ref["a"])
     assert_stage("out", _rows_gpu(case.out, rows), ref["out"])
 
 

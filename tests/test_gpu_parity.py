@@ -117,21 +117,43 @@ def _bf16_ulp(r):
 
 def test_tiny_stages_vs_faithful_oracle(tiny):
     """Against the oracle's diagnostic mode that rounds to bf16 where the GPU
-    stores bf16 (SURVEY reading c23): the fp32 arithmetic of the norm and of
-    the QKV GEMM + QK-norm + RoPE epilogue differs from fp64 by far less than
-    one bf16 spacing, so the stored h1, q, k and v can differ from the rounded
-    fp64 values only where a value sits next to a rounding boundary: at most
-    one spacing, and rarely (>= 99 % identical)."""
+    stores bf16 (SURVEY reading c23), h1 from the inputs and q, k, v from the
+    GPU's h1: the fp32 arithmetic of the norm and of the QKV GEMM + QK-norm +
+    RoPE epilogue is off from fp64 by far less than
+    one bf16 spacing of an O(1) value (fp32 sums of a few hundred products,
+    and the hardware sine / cosine at about 2^-21 absolute), so the stored
+    h1, q, k and v can differ from the rounded fp64 values only where a value
+    sits next to a rounding boundary: by at most one spacing plus that
+    absolute error (which matters only for values near zero, where the
+    rotation cancels), and rarely (>= 99 % identical)."""
     case, _ = tiny
     inp = case.inp
     lay = inp.layout
-    rf = orc.BlockOracle(inp.dims, inp.weights, faithful=True).forward(inp.x, lay.tag, lay.tidx, lay.pos, inp.table)
+    ob = orc.BlockOracle(inp.dims, inp.weights, faithful=True)
+    rf = ob.forward(inp.x, lay.tag, lay.tidx, lay.pos, inp.table)
+    # q, k, v from the GPU's own h1: a legitimate one-spacing difference in
+    # an h1 value moves every q of its row by far more than a q spacing
+    h1_g = case.stage("H1")
+    rq = ob.qkv(to64(h1_g), lay.pos)
     q, k, v = case.qkv()
-    for name, g, f in (("h1", case.stage("H1"), rf["h1"]), ("q", q, rf["q"]), ("k", k, rf["k"]), ("v", v, rf["v"])):
+    d_ = inp.dims
+    ang = orc.rope_angles(lay.pos, d_.rope_pairs, d_.rope_theta, d_.head_dim)     # [N, D/2]
+    for name, g, f in (("h1", h1_g, rf["h1"]), ("q", q, rq["q"]), ("k", k, rq["k"]), ("v", v, rq["v"])):
         g, f = to64(g), to64(f)
         d = np.abs(g - f)
         same = float(np.mean(d == 0))
-        assert np.all(d <= _bf16_ulp(f) * (1 + 1e-12)), f"{name}: a value more than one bf16 spacing off"
+        bound = _bf16_ulp(f) + 2.0 ** -16
+        if name in ("q", "k"):
+            # the rotary angle pos * freq is formed in fp32 (relative error
+            # 2^-23) and its sine / cosine carry about 2^-21 absolute: a pair of
+            # norm r moves by up to r (|angle| 2^-22 + 2^-20)
+            pair = np.sqrt(f[..., 0::2] ** 2 + f[..., 1::2] ** 2)
+            slack = pair * (np.abs(ang)[:, None, :] * 2.0 ** -22 + 2.0 ** -20)
+            bound = bound + np.repeat(slack, 2, axis=-1)
+        bad = np.argwhere(d > bound)
+        detail = [(tuple(int(i) for i in b), float(g[tuple(b)]), float(f[tuple(b)]), float(bound[tuple(b)]))
+                  for b in bad[:4]]
+        assert bad.size == 0, f"{name}: {len(bad)} values more than one bf16 spacing off: {detail}"
         assert same >= 0.99, f"{name}: only {same:.4f} identical to the faithful oracle"
 
 
