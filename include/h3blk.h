@@ -474,16 +474,6 @@ H3BLK_API int h3blk_attention_noalloc_check(void* stream, int* status);
  * reset by the call. INVALID_ARG for a null pointer or a limit out of range. */
 H3BLK_API int h3blk_selftest_wait(int complete, int limit_ms, void* word, void* stream, int* status);
 
-/* Test-only: y[i] = the polynomial 2^x[i] that the attention kernel
- * evaluates on the FMA pipe for a share of its softmax exponentials (2^n by
- * exponent-field addition times a degree-3 fit of 2^f on [-1/2, 1/2]; inputs
- * below -125 are clamped to -125). x and y are caller-owned device fp32 [n],
- * asynchronous on `stream`. Stated error: relative <= 1e-4 for x in
- * [-125, 8]. INVALID_ARG for null pointers or n outside [1, 2^30]. The
- * softmax of "MiniMaxH3Transformer3DModel" (full self-attention) is where it
- * is used. */
-H3BLK_API int h3blk_selftest_exp2(const float* x, float* y, int64_t n, void* stream);
-
 /* Message for a status code (static storage). */
 H3BLK_API const char* h3blk_error_string(int status);
 

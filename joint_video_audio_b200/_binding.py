@@ -33,7 +33,7 @@ EXPORTS = ["h3blk_create", "h3blk_destroy", "h3blk_workspace_bytes", "h3blk_stag
            "h3blk_model_graph_create", "h3blk_graph_launch", "h3blk_graph_info", "h3blk_graph_destroy",
            "h3blk_ulysses_buffer_bytes", "h3blk_ulysses_workspace_bytes", "h3blk_ulysses_qkv",
            "h3blk_ulysses_attention", "h3blk_ulysses_out", "h3blk_set_attention_density",
-           "h3blk_selftest_wait", "h3blk_selftest_exp2", "h3blk_set_debug_accumulators"]
+           "h3blk_selftest_wait", "h3blk_set_debug_accumulators"]
 
 H3BLK_MAX_RANKS = 8
 
@@ -123,7 +123,6 @@ def _load():
         "h3blk_attention_noalloc": (i32, [i64, i32, i32, i32, i32, vp, vp, vp, vp, vp]),
         "h3blk_attention_noalloc_check": (i32, [vp, C.POINTER(i32)]),
         "h3blk_selftest_wait": (i32, [i32, i32, vp, vp, C.POINTER(i32)]),
-        "h3blk_selftest_exp2": (i32, [vp, vp, i64, vp]),
         "h3blk_set_debug_accumulators": (i32, [vp, i32, vp, C.c_size_t]),
         "h3blk_modulation_scratch_bytes": (i32, [vp, C.POINTER(h3blk_mod_weights), C.POINTER(sz)]),
         "h3blk_modulation_table": (i32, [vp, C.POINTER(h3blk_mod_weights), C.POINTER(C.c_float),
@@ -283,12 +282,6 @@ def h3blk_set_debug_accumulators(handle, gemm: int, buf, nbytes: int) -> None:
     """Test-only (W8A8): later forwards also dump int8 GEMM `gemm`'s raw int32
     accumulators (0 QKV, 1 out-proj, 2 FFN up, 3 FFN down; -1 off) to `buf`."""
     _check("h3blk_set_debug_accumulators", _lib.h3blk_set_debug_accumulators(handle, gemm, buf, nbytes))
-
-
-def h3blk_selftest_exp2(x, y, n, stream) -> None:
-    """Test-only: y = the attention's FMA-pipe polynomial 2^x (device fp32
-    pointers, n elements)."""
-    _check("h3blk_selftest_exp2", _lib.h3blk_selftest_exp2(x, y, n, stream))
 
 
 def h3blk_modulation_scratch_bytes(handle, w: h3blk_mod_weights) -> int:

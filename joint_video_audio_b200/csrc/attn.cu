@@ -73,7 +73,6 @@ constexpr int kSoftmaxWarps = 8;
 constexpr int kThreads = 32 * (2 + kSoftmaxWarps);
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;
-constexpr int kPolyEvery = 4;  // one exponential pair in four on the FMA pipe
 
 template <int D>
 struct AttnSmem {
@@ -405,13 +404,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       const float m_use = grow ? m_new : m_run;
       const float m_sub = m_use == -CUDART_INF_F ? 0.f : m_use;
       const float alpha = grow ? ex2_approx(m_run - m_use) : 1.f;
-      // exponentials on pairs: x = s * scale - m with one packed FMA; one pair
-      // in kPolyEvery goes through the FMA-pipe polynomial, the rest through
-      // the MUFU, so both units share the load. Each half of P (keys 0..63,
-      // then 64..127) is packed to bf16 pairs, stored over the first 64
-      // columns of this tile's S and announced on its own barrier, so the
-      // P V product starts on the first half while the second is computed.
-      // The row sum runs in two packed accumulators.
+      // exponentials on pairs: x = s * scale - m with one packed FMA, then
+      // the MUFU's 2^x (measured: the exponentials are not on this kernel's
+      // critical path, so none are moved to the FMA pipe). Each half of P
+      // (keys 0..63, then 64..127) is packed to bf16 pairs, stored over the
+      // first 64 columns of this tile's S and announced on its own barrier, so
+      // the P V product starts on the first half while the second is
+      // computed. The row sum runs in two packed accumulators.
       const uint64_t sc2 = f2_pack(scale_log2, scale_log2), nm2 = f2_pack(-m_sub, -m_sub);
       uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = acc0;
 #pragma unroll
@@ -423,11 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
           const int cg = 64 * h + c;  // column within the tile
           float x0, x1;
           f2_unpack(f2_fma(f2_pack(sv[c], sv[c + 1]), sc2, nm2), x0, x1);
-          uint64_t e;
-          if (((cg >> 1) % kPolyEvery) == kPolyEvery - 1)
-            e = f2_exp2_poly(x0, x1);
-          else
-            e = f2_pack(ex2_approx(x0), ex2_approx(x1));
+          const uint64_t e = f2_pack(ex2_approx(x0), ex2_approx(x1));
           if ((cg >> 1) & 1)
             acc1 = f2_add(acc1, e);
           else

@@ -326,36 +326,6 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return d;
 }
 
-// 2^x for a pair of floats on the FMA and integer pipes instead of the MUFU:
-// Cody-Waite style split x = n + f with n = round(x) (obtained by adding
-// 1.5 * 2^23, which leaves n in the low mantissa bits) and f in [-1/2, 1/2];
-// 2^f from a degree-3 polynomial fitted here for minimal relative error on
-// [-1/2, 1/2] (Lawson's iteratively reweighted least squares; max relative
-// error 7.5e-5); then n is added to the exponent field. Inputs are clamped to
-// [-125, +inf) so the exponent stays normal; callers keep x <= 8.
-__device__ __forceinline__ uint64_t f2_exp2_poly(float x0, float x1) {
-  x0 = fmaxf(x0, -125.f);
-  x1 = fmaxf(x1, -125.f);
-  const uint64_t x = f2_pack(x0, x1);
-  const uint64_t magic = f2_pack(12582912.f, 12582912.f);
-  const uint64_t nmagic = f2_pack(-12582912.f, -12582912.f);
-  const uint64_t j = f2_add(x, magic);
-  const uint64_t n = f2_add(j, nmagic);
-  const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), x);
-  uint64_t p = f2_fma(f, f2_pack(0.0551716648042202f, 0.0551716648042202f),
-                      f2_pack(0.2426111251115799f, 0.2426111251115799f));
-  p = f2_fma(p, f, f2_pack(0.6932609677314758f, 0.6932609677314758f));
-  p = f2_fma(p, f, f2_pack(0.9999280571937561f, 0.9999280571937561f));
-  uint32_t p0, p1, j0, j1;
-  asm("mov.b64 {%0, %1}, %2;" : "=r"(p0), "=r"(p1) : "l"(p));
-  asm("mov.b64 {%0, %1}, %2;" : "=r"(j0), "=r"(j1) : "l"(j));
-  p0 += j0 << 23;
-  p1 += j1 << 23;
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(p0), "r"(p1));
-  return r;
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

@@ -42,32 +42,3 @@ extern "C" int h3blk_selftest_wait(int complete, int limit_ms, void* word, void*
   *status = (bits & h3::kErrTimeoutStream) ? H3BLK_ERR_TIMEOUT : H3BLK_OK;
   return H3BLK_OK;
 }
-
-// h3blk_selftest_exp2: evaluates, element by element, the polynomial 2^x that
-// the attention kernel runs on the FMA pipe for a share of its softmax
-// exponentials (f2_exp2_poly in ptx.cuh), so that a test can hold it to its
-// stated error bound against an exact 2^x.
-namespace {
-
-__global__ void exp2_selftest_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t n) {
-  const int64_t i = 2 * (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x);
-  if (i >= n) return;
-  const float a = x[i];
-  const float b = (i + 1 < n) ? x[i + 1] : 0.f;
-  const uint64_t r = h3::f2_exp2_poly(a, b);
-  uint32_t r0, r1;
-  asm("mov.b64 {%0, %1}, %2;" : "=r"(r0), "=r"(r1) : "l"(r));
-  y[i] = __uint_as_float(r0);
-  if (i + 1 < n) y[i + 1] = __uint_as_float(r1);
-}
-
-}  // namespace
-
-extern "C" int h3blk_selftest_exp2(const float* x, float* y, int64_t n, void* stream) {
-  if (!x || !y || n < 1 || n > (int64_t(1) << 30)) return H3BLK_ERR_INVALID_ARG;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const int threads = 256;
-  const int64_t blocks = ((n + 1) / 2 + threads - 1) / threads;
-  exp2_selftest_kernel<<<static_cast<unsigned>(blocks), threads, 0, s>>>(x, y, n);
-  return cudaGetLastError() == cudaSuccess ? H3BLK_OK : H3BLK_ERR_CUDA;
-}

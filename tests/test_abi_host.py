@@ -410,11 +410,5 @@ def test_debug_accumulator_dump_validation():
     assert lib.h3blk_set_debug_accumulators(None, -1, None, 0) == B.H3BLK_ERR_INVALID_ARG
 
 
-@pytest.mark.parametrize("args", [(0, 0, 1, 0), (1 << 20, 0, 4, 0), (0, 1 << 20, 4, 0), (1 << 20, 1 << 21, 0, 0),
-                                  (1 << 20, 1 << 21, (1 << 30) + 1, 0)])
-def test_selftest_exp2_validates_before_gpu(args):
-    assert B._lib.h3blk_selftest_exp2(*args) == B.H3BLK_ERR_INVALID_ARG
-
-
 def test_noalloc_check_validates_status_pointer():
     assert B._lib.h3blk_attention_noalloc_check(None, None) == B.H3BLK_ERR_INVALID_ARG
