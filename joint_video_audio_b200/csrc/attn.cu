@@ -146,6 +146,21 @@ struct KvSeq {
   }
 };
 
+// Non-blocking look at a barrier phase: true if the phase of parity
+// `parity` has completed. Several can be in flight at once, so the issuer
+// pays one barrier latency for a batch of checks instead of one per check.
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 __device__ __forceinline__ void fail(int* err, volatile int* abort) {
   if (err) atomicOr(err, kErrTimeoutAttn);
   *abort = 1;
@@ -274,12 +289,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       // TMEM columns [t*128, t*128 + 64), 8 columns per K = 16 step
       // Each half of P (keys 0..63, 64..127) has its own ready barrier, so the
       // first four K steps run while the softmax still works on the second half.
-      auto issue_pv = [&](int t, int j, int vslot) -> bool {
+      auto issue_pv = [&](int t, int j, int vslot, bool lo_seen) -> bool {
         const uint64_t vd = vdesc0 + (uint64_t)((vslot * SM::kKVBytes) >> 4);
         const uint32_t dtm = tmem + 256 + t * kTile, atm = tmem + t * kTile;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          if (!mbar_wait(half == 0 ? &s.p_lo[t] : &s.p_hi[t], j & 1, abort)) return false;
+          if (!(half == 0 && lo_seen) && !mbar_wait(half == 0 ? &s.p_lo[t] : &s.p_hi[t], j & 1, abort)) return false;
           tc_fence_after();
 #pragma unroll
           for (int kk = 4 * half; kk < 4 * half + 4; ++kk)
@@ -295,15 +310,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         if (ok) mma_commit(&s.ring_empty[0]);
         RingPos vpos{1, 0u}, kpos{2 % kSlots, 2 >= kSlots ? 1u : 0u};  // V_j and K_{j+1}
         for (int j = 0; ok && j < n_kv; ++j) {
-          // the ring waits come first: they are normally satisfied long before
-          // P, and polling them between P V and the next S would put their
-          // latency on the critical path
+          // The tensor pipe queues only two or three products, so every
+          // barrier latency this thread sits through while the queue is empty
+          // is tensor idle time: the ring slots of V_j and K_{j+1} and the
+          // first half of P_0 are looked at in one batch (the latencies
+          // overlap), with a blocking wait only for what is not complete yet;
+          // the look at P_1 is answered while S_0 issues.
           const bool more = j + 1 < n_kv;
-          ok = wait_ring(vpos) && (!more || wait_ring(kpos)) && issue_pv(0, j, vpos.slot);
+          const bool tv = mbar_test(&s.ring_full[vpos.slot], vpos.phase);
+          const bool tk = !more || mbar_test(&s.ring_full[kpos.slot], kpos.phase);
+          const bool tp0 = mbar_test(&s.p_lo[0], j & 1);
+          ok = (tv || wait_ring(vpos)) && (tk || wait_ring(kpos)) && issue_pv(0, j, vpos.slot, tp0);
           if (!ok) break;
+          const bool tp1 = mbar_test(&s.p_lo[1], j & 1);  // answered while S0 issues
           if (more) ok = issue_s(0, kpos.slot);
           if (!ok) break;
-          ok = issue_pv(1, j, vpos.slot);
+          ok = issue_pv(1, j, vpos.slot, tp1);
           if (!ok) break;
           mma_commit(&s.ring_empty[vpos.slot]);
           if (more) {
