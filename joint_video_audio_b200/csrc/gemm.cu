@@ -11,6 +11,12 @@
 // epilogue of tile i overlaps the main loop of tile i+1. Operands are staged by
 // TMA with the 128-byte swizzle the UMMA descriptors expect.
 //
+// Two kernels share these roles and epilogues: gemm_pair_kernel (used on
+// B200) runs on clusters of two CTAs with 256 x 256 cluster tiles and
+// products of M = 256 spanning both SMs (each SM stages its own 128 rows of A
+// and half of B's rows: a third less shared-memory operand traffic per SM,
+// six stages); gemm_kernel is the single-CTA form.
+//
 // Fused epilogues (sources: "MiniMaxH3Transformer3DModel", diffusers API
 // page, constructor: qk_norm_eps of the per-head query/key norms, rope_theta;
 // introduction: AdaLN modulation per modality tag; ffn_dim of the SwiGLU):
@@ -45,6 +51,7 @@ constexpr int kEpiWarps = 8;  // two per TMEM lane quadrant, each on one half of
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kTmemCols = 512;  // two 256-column fp32 accumulators
 constexpr int kGroupN = 8;      // tile raster: 8 N-tiles share each pass over M
+constexpr int kGroupNPair = 12; // the CTA-pair kernel's raster (measured best of 4, 8, 12, 16)
 constexpr size_t kSmemBytes = 1024 + (size_t)kStages * (kAStage + kBStage) + 256;
 
 struct Smem {
@@ -81,11 +88,12 @@ struct TileCoord {
   int m, n;
 };
 
+template <int GROUP = kGroupN>
 __device__ __forceinline__ TileCoord tile_coord(int t, int tiles_m, int tiles_n) {
-  const int group = t / (kGroupN * tiles_m);
-  const int first_n = group * kGroupN;
-  const int gn = min(kGroupN, tiles_n - first_n);
-  const int idx = t - group * kGroupN * tiles_m;
+  const int group = t / (GROUP * tiles_m);
+  const int first_n = group * GROUP;
+  const int gn = min(GROUP, tiles_n - first_n);
+  const int idx = t - group * GROUP * tiles_m;
   return {idx / gn, first_n + idx % gn};
 }
 
@@ -463,6 +471,233 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
 }
 
+// ------------------------------------------------------------------ CTA-pair kernel
+// The same GEMM on clusters of two CTAs (one per SM of a pair): a cluster
+// tile is 256 x 256; each CTA stages its 128 rows of A and its 128 rows of B
+// (the weight rows of one half of the tile's columns), and the pair's first
+// CTA issues products of M = 256, N = 256 that read A and B from both SMs'
+// shared memory and leave each SM's 128 rows of the accumulator in its own
+// tensor memory. Per SM that is the single-CTA kernel's 128 x 256 tile with
+// two thirds of its shared-memory operand traffic (B is split, not
+// duplicated), so more stages fit. Both CTAs' loads signal the first CTA's
+// "full" barrier; the issuer's commits arrive on the "empty", "accumulator
+// full" and final barriers of both CTAs; the second CTA's epilogue warps
+// release an accumulator buffer on the first CTA's barrier.
+constexpr int kStagesPair = 6;
+constexpr int kBHalfStage = 128 * kRowBytes;  // 16 KB
+constexpr size_t kSmemBytesPair = 1024 + (size_t)kStagesPair * (kAStage + kBHalfStage) + 256;
+
+struct SmemPair {
+  uint8_t* a;
+  uint8_t* b;
+  uint64_t* full;
+  uint64_t* empty;
+  uint64_t* tfull;
+  uint64_t* tempty;
+  uint64_t* drain;
+  uint32_t* tmem_base;
+  int* abort;
+};
+
+__device__ __forceinline__ SmemPair carve_pair(uint8_t* raw) {
+  const uint32_t base = smem_u32(raw);
+  const uint32_t pad = ((base + 1023u) & ~1023u) - base;
+  uint8_t* p = raw + pad;
+  SmemPair s;
+  s.a = p;
+  s.b = p + kStagesPair * kAStage;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(p + kStagesPair * (kAStage + kBHalfStage));
+  s.full = bars;
+  s.empty = bars + kStagesPair;
+  s.tfull = bars + 2 * kStagesPair;
+  s.tempty = bars + 2 * kStagesPair + 2;
+  s.drain = bars + 2 * kStagesPair + 4;
+  s.tmem_base = reinterpret_cast<uint32_t*>(bars + 2 * kStagesPair + 5);
+  s.abort = reinterpret_cast<int*>(bars + 2 * kStagesPair + 6);
+  return s;
+}
+
+__device__ __forceinline__ void fail_pair(const SmemPair& s, int* err) {
+  if (err) atomicOr(err, kErrTimeoutGemm);
+  *reinterpret_cast<volatile int*>(s.abort) = 1;
+}
+
+template <int EPI, bool INT8>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const GemmArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  const SmemPair s = carve_pair(smem_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int cluster = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
+  const int tiles_m = (int)((p.M + 2 * BM - 1) / (2 * BM));
+  const int tiles_n = EPI == kEpiSwiGLU ? p.N / 128 : (p.N + BN - 1) / BN;
+  const int num_tiles = tiles_m * tiles_n;
+  const int num_kb = p.K / (INT8 ? 128 : 64);
+  volatile int* abort = s.abort;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStagesPair; ++i) {
+      mbar_init(&s.full[i], 1);   // the first CTA's producer arrives; both CTAs' bytes complete it
+      mbar_init(&s.empty[i], 1);  // one commit of the issuer
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.tfull[i], 1);
+      mbar_init(&s.tempty[i], 2 * kEpiWarps);  // every epilogue warp of both CTAs
+    }
+    mbar_init(s.drain, 1);
+    *s.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(s.tmem_base, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  // both CTAs' barriers are initialised and their tensor memory allocated
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *s.tmem_base;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer (both CTAs)
+    if (lane == 0) {
+      const uint32_t full0 = mapa_shared(smem_u32(s.full), 0);  // the first CTA's full barriers
+      int stage = 0;
+      uint32_t phase = 0;
+      long issued = 0;
+      bool ok = true;
+      for (int t = cluster; t < num_tiles && ok; t += n_clusters) {
+        const TileCoord tc = tile_coord<kGroupNPair>(t, tiles_m, tiles_n);
+        const int ya = tc.m * 2 * BM + (int)rank * BM;
+        const int yb = EPI == kEpiSwiGLU ? (rank == 0 ? tc.n * 128 : p.N + tc.n * 128) : tc.n * BN + (int)rank * 128;
+        // A box wholly past the last row (the second CTA's rows of a short
+        // last M tile) or a B box wholly past the last weight row (the second
+        // half of a last N tile) is not loaded: the accumulator rows / columns
+        // it would feed are never stored. The first CTA's boxes always hold
+        // data, and it expects the bytes of every box the pair loads.
+        const bool a1 = tc.m * 2 * BM + BM < p.M;
+        const bool b1 = EPI == kEpiSwiGLU || tc.n * BN + 128 < p.Nb;
+        const bool load_a = rank == 0 || a1, load_b = rank == 0 || b1;
+        const uint32_t bytes = kAStage + kBHalfStage + (a1 ? kAStage : 0) + (b1 ? kBHalfStage : 0);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&s.empty[stage], phase ^ 1, abort)) {
+            fail_pair(s, p.err);
+            ok = false;
+            break;
+          }
+          const int x = kb * (INT8 ? 128 : 64);
+          if (rank == 0) mbar_expect_tx(&s.full[stage], bytes);
+          if (load_a) tma_load_2d_pair(s.a + stage * kAStage, &tmA, full0 + 8u * stage, x, ya);
+          if (load_b) tma_load_2d_pair(s.b + stage * kBHalfStage, &tmB, full0 + 8u * stage, x, yb);
+          ++issued;
+          if (++stage == kStagesPair) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      // Drain (first CTA; its full barriers count both CTAs' bytes): the last
+      // loads issued must have landed before either CTA exits.
+      if (rank == 0) {
+        const long outstanding = issued < kStagesPair ? issued : kStagesPair;
+        for (long i = 0; i < outstanding; ++i) {
+          if (--stage < 0) {
+            stage = kStagesPair - 1;
+            phase ^= 1;
+          }
+          mbar_wait(&s.full[stage], phase, nullptr);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer (first CTA)
+    if (lane == 0 && rank == 0) {
+      const uint32_t idesc = INT8 ? make_idesc(2, 1, 2 * BM, BN, false) : make_idesc(1, 1, 2 * BM, BN, false);
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      bool ok = true;
+      for (int t = cluster; t < num_tiles && ok; t += n_clusters, ++local) {
+        const int buf = local & 1;
+        const uint32_t use = (uint32_t)(local >> 1);
+        if (!mbar_wait(&s.tempty[buf], (use & 1) ^ 1, abort)) {
+          fail_pair(s, p.err);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem_base + buf * BN;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&s.full[stage], phase, abort)) {
+            fail_pair(s, p.err);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(s.a + stage * kAStage);
+          const uint32_t b0 = smem_u32(s.b + stage * kBHalfStage);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint64_t ad = sw128_desc(a0 + k * 32, 16);
+            const uint64_t bd = sw128_desc(b0 + k * 32, 16);
+            if (INT8)
+              mma_s8_ss_pair(d, ad, bd, idesc, (kb | k) != 0);
+            else
+              mma_bf16_ss_pair(d, ad, bd, idesc, (kb | k) != 0);
+          }
+          mma_commit_pair(&s.empty[stage], 0x3);
+          if (++stage == kStagesPair) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (ok) mma_commit_pair(&s.tfull[buf], 0x3);
+      }
+      // every product issued has completed once `drain` flips (in both CTAs)
+      mma_commit_pair(s.drain, 0x3);
+      mbar_wait(s.drain, 0, nullptr);
+    } else if (lane == 0) {
+      // second CTA: its shared memory and tensor memory serve the pair's
+      // products until the last one completes
+      mbar_wait(s.drain, 0, nullptr);
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue (both CTAs)
+    const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const uint32_t tempty0 = mapa_shared(smem_u32(s.tempty), 0);
+    int local = 0;
+    for (int t = cluster; t < num_tiles; t += n_clusters, ++local) {
+      const TileCoord tc = tile_coord<kGroupNPair>(t, tiles_m, tiles_n);
+      const int buf = local & 1;
+      const uint32_t use = (uint32_t)(local >> 1);
+      if (!mbar_wait(&s.tfull[buf], use & 1, abort)) {
+        if (lane == 0) fail_pair(s, p.err);
+        break;
+      }
+      tc_fence_after();
+      const int64_t row = (int64_t)tc.m * 2 * BM + (int64_t)rank * BM + quad * 32 + lane;
+      const uint32_t tacc = tmem_base + ((uint32_t)(quad * 32) << 16) + buf * BN;
+      epilogue_tile<EPI, INT8>(p, tacc, row, row < p.M, tc.n, half);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty0 + 8u * buf);
+    }
+  }
+
+  // neither CTA leaves while the other may still signal its barriers or read
+  // its memory
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem_base, kTmemCols);
+}
+
 CUresult make_map(PFN_cuTensorMapEncodeTiled_v12000 encode, CUtensorMap* m, const void* ptr, uint64_t rows,
                   uint64_t cols, bool int8) {
   const CUtensorMapDataType dt = int8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -488,6 +723,32 @@ cudaError_t launch_t(const GemmArgs& a, const CUtensorMap& ta, const CUtensorMap
   return cudaGetLastError();
 }
 
+template <int EPI, bool INT8>
+cudaError_t launch_pair_t(const GemmArgs& a, const CUtensorMap& ta, const CUtensorMap& tb, int num_sms,
+                          cudaStream_t s) {
+  auto k = gemm_pair_kernel<EPI, INT8>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytesPair);
+  if (e != cudaSuccess) return e;
+  const int tiles_m = (int)((a.M + 2 * BM - 1) / (2 * BM));
+  const int tiles_n = EPI == kEpiSwiGLU ? a.N / 128 : (a.N + BN - 1) / BN;
+  const long tiles = (long)tiles_m * tiles_n;
+  const int max_clusters = num_sms / 2;
+  const int clusters = (int)(tiles < max_clusters ? tiles : max_clusters);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * clusters);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytesPair;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k, ta, tb, a);
+}
+
 }  // namespace
 
 cudaError_t launch_gemm(const GemmArgs& a, PFN_cuTensorMapEncodeTiled_v12000 encode, int num_sms, cudaStream_t s) {
@@ -499,6 +760,28 @@ cudaError_t launch_gemm(const GemmArgs& a, PFN_cuTensorMapEncodeTiled_v12000 enc
   CUtensorMap ta, tb;
   if (make_map(encode, &ta, a.A, (uint64_t)a.M, (uint64_t)a.K, a.int8) != CUDA_SUCCESS) return cudaErrorInvalidValue;
   if (make_map(encode, &tb, a.B, (uint64_t)a.Nb, (uint64_t)a.K, a.int8) != CUDA_SUCCESS) return cudaErrorInvalidValue;
+#ifndef H3_GEMM_PAIR
+#define H3_GEMM_PAIR 1
+#endif
+  if (H3_GEMM_PAIR && num_sms >= 2) {
+    if (a.int8) {
+      switch (a.epi) {
+        case kEpiStoreBf16: return launch_pair_t<kEpiStoreBf16, true>(a, ta, tb, num_sms, s);
+        case kEpiQKV: return launch_pair_t<kEpiQKV, true>(a, ta, tb, num_sms, s);
+        case kEpiResid: return launch_pair_t<kEpiResid, true>(a, ta, tb, num_sms, s);
+        case kEpiSwiGLU: return launch_pair_t<kEpiSwiGLU, true>(a, ta, tb, num_sms, s);
+        case kEpiStoreS32: return launch_pair_t<kEpiStoreS32, true>(a, ta, tb, num_sms, s);
+      }
+    } else {
+      switch (a.epi) {
+        case kEpiStoreBf16: return launch_pair_t<kEpiStoreBf16, false>(a, ta, tb, num_sms, s);
+        case kEpiQKV: return launch_pair_t<kEpiQKV, false>(a, ta, tb, num_sms, s);
+        case kEpiResid: return launch_pair_t<kEpiResid, false>(a, ta, tb, num_sms, s);
+        case kEpiSwiGLU: return launch_pair_t<kEpiSwiGLU, false>(a, ta, tb, num_sms, s);
+      }
+    }
+    return cudaErrorInvalidValue;
+  }
   if (a.int8) {
     switch (a.epi) {
       case kEpiStoreBf16: return launch_t<kEpiStoreBf16, true>(a, ta, tb, num_sms, s);
