@@ -2,7 +2,8 @@
 // with the block's fused epilogues (K2a/K2b/K2c/K2d, and the int8 K5).
 //
 //   warp 0      TMA producer: A tile 128 x 128 B and B tile 256 x 128 B per stage
-//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
+//   warp 1      TMEM allocator + tcgen05.mma issuer (the whole warp runs the
+//               loop, lane 0 issues)
 //   warps 2..9  epilogue: tcgen05.ld of the fp32 / s32 accumulator (thread =
 //               output row; the two warps of a lane quadrant take one half of
 //               the tile's columns each), fused math, 16-byte global stores
@@ -397,7 +398,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    // the whole warp runs the loop (warp-uniform descriptors); lane 0 issues
+    // every product and commit
+    {
       const uint32_t idesc = INT8 ? make_idesc(2, 1, BM, BN, false) : make_idesc(1, 1, BM, BN, false);
       int stage = 0;
       uint32_t phase = 0;
@@ -406,15 +409,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++local) {
         const int buf = local & 1;
         const uint32_t use = (uint32_t)(local >> 1);
-        if (!mbar_wait(&s.tempty[buf], (use & 1) ^ 1, abort)) {
-          fail(s, p.err);
+        if (!mbar_wait_warp(&s.tempty[buf], (use & 1) ^ 1, abort)) {
+          if (lane == 0) fail(s, p.err);
           break;
         }
         tc_fence_after();
         const uint32_t d = tmem_base + buf * BN;
         for (int kb = 0; kb < num_kb; ++kb) {
-          if (!mbar_wait(&s.full[stage], phase, abort)) {
-            fail(s, p.err);
+          if (!mbar_wait_warp(&s.full[stage], phase, abort)) {
+            if (lane == 0) fail(s, p.err);
             ok = false;
             break;
           }
@@ -426,20 +429,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t ad = sw128_desc(a0 + k * 32, 16);
             const uint64_t bd = sw128_desc(b0 + k * 32, 16);
             if (INT8)
-              mma_s8_ss(d, ad, bd, idesc, (kb | k) != 0);
+              mma_s8_ss_w(d, ad, bd, idesc, (kb | k) != 0);
             else
-              mma_bf16_ss(d, ad, bd, idesc, (kb | k) != 0);
+              mma_bf16_ss_w(d, ad, bd, idesc, (kb | k) != 0);
           }
-          mma_commit(&s.empty[stage]);
+          mma_commit_w(&s.empty[stage]);
           if (++stage == kStages) {
             stage = 0;
             phase ^= 1;
           }
         }
-        if (ok) mma_commit(&s.tfull[buf]);
+        if (ok) mma_commit_w(&s.tfull[buf]);
       }
-      // every MMA issued by this thread has completed once `drain` flips
-      mma_commit(s.drain);
+      // every MMA issued by lane 0 has completed once `drain` flips
+      mma_commit_w(s.drain);
       mbar_wait(s.drain, 0, nullptr);
     }
   } else {
@@ -617,7 +620,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer (first CTA)
-    if (lane == 0 && rank == 0) {
+    // the whole warp runs the loop (warp-uniform descriptors); lane 0 issues
+    // every product and commit
+    if (rank == 0) {
       const uint32_t idesc = INT8 ? make_idesc(2, 1, 2 * BM, BN, false) : make_idesc(1, 1, 2 * BM, BN, false);
       int stage = 0;
       uint32_t phase = 0;
@@ -626,15 +631,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = cluster; t < num_tiles && ok; t += n_clusters, ++local) {
         const int buf = local & 1;
         const uint32_t use = (uint32_t)(local >> 1);
-        if (!mbar_wait(&s.tempty[buf], (use & 1) ^ 1, abort)) {
-          fail_pair(s, p.err);
+        if (!mbar_wait_warp(&s.tempty[buf], (use & 1) ^ 1, abort)) {
+          if (lane == 0) fail_pair(s, p.err);
           break;
         }
         tc_fence_after();
         const uint32_t d = tmem_base + buf * BN;
         for (int kb = 0; kb < num_kb; ++kb) {
-          if (!mbar_wait(&s.full[stage], phase, abort)) {
-            fail_pair(s, p.err);
+          if (!mbar_wait_warp(&s.full[stage], phase, abort)) {
+            if (lane == 0) fail_pair(s, p.err);
             ok = false;
             break;
           }
@@ -646,20 +651,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t ad = sw128_desc(a0 + k * 32, 16);
             const uint64_t bd = sw128_desc(b0 + k * 32, 16);
             if (INT8)
-              mma_s8_ss_pair(d, ad, bd, idesc, (kb | k) != 0);
+              mma_s8_ss_pair_w(d, ad, bd, idesc, (kb | k) != 0);
             else
-              mma_bf16_ss_pair(d, ad, bd, idesc, (kb | k) != 0);
+              mma_bf16_ss_pair_w(d, ad, bd, idesc, (kb | k) != 0);
           }
-          mma_commit_pair(&s.empty[stage], 0x3);
+          mma_commit_pair_w(&s.empty[stage], 0x3);
           if (++stage == kStagesPair) {
             stage = 0;
             phase ^= 1;
           }
         }
-        if (ok) mma_commit_pair(&s.tfull[buf], 0x3);
+        if (ok) mma_commit_pair_w(&s.tfull[buf], 0x3);
       }
       // every product issued has completed once `drain` flips (in both CTAs)
-      mma_commit_pair(s.drain, 0x3);
+      mma_commit_pair_w(s.drain, 0x3);
       mbar_wait(s.drain, 0, nullptr);
     } else if (lane == 0) {
       // second CTA: its shared memory and tensor memory serve the pair's
