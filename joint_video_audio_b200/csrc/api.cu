@@ -83,6 +83,7 @@ struct Layout {
   size_t len[H3BLK_STAGE_COUNT];
   size_t tiles_off;
   size_t modt_off;
+  size_t rope_off;
   size_t sp_qsum, sp_ksum, sp_count;  // block-sparse pooling buffers (0 when dense)
   size_t total;
 };
@@ -103,6 +104,8 @@ Layout make_layout(const h3blk_config& c, int64_t n, int keep_per_1024) {
   const bool q = c.quant != 0;
   L.modt_off = o;
   if (q) o = align256(o + h3::modt_bytes(c.n_tags, c.n_t, c.hidden));
+  L.rope_off = o;
+  o = align256(o + h3::rope_table_bytes(n, c.head_dim / 2));
   if (!q) put(H3BLK_STAGE_H1, N * C * 2);
   put(H3BLK_STAGE_QKV, N * 3 * HD * 2);
   put(H3BLK_STAGE_O, N * HD * 2);
@@ -267,7 +270,6 @@ int phase_qkv(const h3blk_ctx* h, const Span& sp, const void* x, const int32_t* 
   g.ld_out = 3 * HD;
   g.q_gain = static_cast<const __nv_bfloat16*>(w->q_gain);
   g.k_gain = static_cast<const __nv_bfloat16*>(w->k_gain);
-  g.pos = pos + 3 * sp.row0;
   g.s_a = q ? b.h1_s : nullptr;
   g.s_b = w->s_qkv;
   if (route) {
@@ -276,8 +278,10 @@ int phase_qkv(const h3blk_ctx* h, const Span& sp, const void* x, const int32_t* 
     g.route_row0 = sp.row0;
     for (int r = 0; r < route->ranks; ++r) g.route_dst[r] = route->dst[r];
   }
+  g.rope_tab = b.rope_tab;
   if (int st = attach_dump(h, 0, g)) return st;
   H3_TRY(mark(h, timing, 2, s));
+  H3_TRY(h3::launch_rope_table(pos + 3 * sp.row0, sp.n_local, h->rope, c.head_dim / 2, b.rope_tab, s));
   H3_TRY(h3::launch_gemm(g, enc, sms, s));
   return H3BLK_OK;
 }
@@ -437,6 +441,7 @@ int block_forward(const h3blk_ctx* h, int64_t n_rows, const void* x, const int32
   b.err = reinterpret_cast<int*>(buf(H3BLK_STAGE_ERROR));
   b.tiles = reinterpret_cast<h3::TileInfo*>(ws + L.tiles_off);
   b.modt = reinterpret_cast<float4*>(ws + L.modt_off);
+  b.rope_tab = reinterpret_cast<float2*>(ws + L.rope_off);
   const bool sparse = h->keep_per_1024 < 1024;
   b.sp_qsum = sparse ? reinterpret_cast<float*>(ws + L.sp_qsum) : nullptr;
   b.sp_ksum = sparse ? reinterpret_cast<float*>(ws + L.sp_ksum) : nullptr;

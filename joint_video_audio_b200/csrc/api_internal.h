@@ -40,6 +40,7 @@ struct BlockBufs {
   int* err = nullptr;
   h3::TileInfo* tiles = nullptr;
   float4* modt = nullptr;  // the pre-norm vectors rearranged for the row passes
+  float2* rope_tab = nullptr;  // (sin, cos) of this call's rows' rotary angles, [rows, head_dim / 2]
   // block-sparse selection (null when dense)
   float *sp_qsum = nullptr, *sp_ksum = nullptr;
   int32_t *sp_count = nullptr, *sp_lists = nullptr;

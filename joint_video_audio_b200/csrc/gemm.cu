@@ -22,7 +22,8 @@
 // page, constructor: qk_norm_eps of the per-head query/key norms, rope_theta;
 // introduction: AdaLN modulation per modality tag; ffn_dim of the SwiGLU):
 //   kEpiQKV    q, k: per-head RMSNorm (fp32) * gain, then 3D RoPE on adjacent
-//              pairs; v: stored as is. Output [M, 3*H*D] bf16, or, routed by
+//              pairs, the (sin, cos) of each row's angles read from a table
+//              made once per forward (rope_table_kernel); v: stored as is. Output [M, 3*H*D] bf16, or, routed by
 //              head group for sequence parallelism, each head's q / k / v to
 //              its group owner's [rows, 3*Hg*D] buffer (peer memory or a send
 //              buffer).
@@ -153,6 +154,19 @@ __device__ __forceinline__ void rope_sincos(float x, float& sn, float& cs) {
   __sincosf(r, &sn, &cs);
 }
 
+// One thread per (row, pair): the table the QKV epilogue reads.
+__global__ void rope_table_kernel(const int32_t* __restrict__ pos, int64_t n, const RopeTable rope, int pairs,
+                                  float2* __restrict__ tab) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n * pairs) return;
+  const int64_t row = i / pairs;
+  const int pair = (int)(i - row * pairs);
+  const int ax = rope.axis[pair];
+  float sn = 0.f, cs = 1.f;
+  if (ax < 3) rope_sincos((float)__ldg(pos + row * 3 + ax) * rope.freq[pair], sn, cs);
+  tab[i] = make_float2(sn, cs);
+}
+
 // ------------------------------------------------------------------ epilogue
 template <int EPI, bool INT8>
 __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tacc, int64_t row, bool row_ok, int n_tile,
@@ -240,12 +254,6 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tacc, 
   }
   if (EPI == kEpiQKV) {
     const int D = p.head_dim;
-    int pos3[3] = {0, 0, 0};
-    if (row_ok) {
-      pos3[0] = __ldg(p.pos + row * 3 + 0);
-      pos3[1] = __ldg(p.pos + row * 3 + 1);
-      pos3[2] = __ldg(p.pos + row * 3 + 2);
-    }
     const int heads_per_half = (BN / 2) / D;
 #pragma unroll 1
     for (int hh = half * heads_per_half; hh < (half + 1) * heads_per_half; ++hh) {
@@ -285,18 +293,25 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tacc, 
       const __nv_bfloat16* gain = region == 0 ? p.q_gain : p.k_gain;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
+        // this chunk's 16 (sin, cos) pairs, requested before the accumulators
+        float4 sc[8];
+        if (row_ok) {
+          const float4* t4 = reinterpret_cast<const float4*>(p.rope_tab + row * (D / 2) + c * 16);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) sc[i] = __ldg(t4 + i);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) sc[i] = make_float4(0.f, 1.f, 0.f, 1.f);
+        }
         float v[32];
         load_chunk<INT8>(th + c * 32, sa, p.s_b, col0 + c * 32, v, dump);
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = v[j] * rstd * __bfloat162float(gain[c * 32 + j]);
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
-          const int pair = c * 16 + q;
-          const int ax = p.rope.axis[pair];
-          if (ax < 3) {
-            float sn, cs;
-            const int pv = ax == 0 ? pos3[0] : (ax == 1 ? pos3[1] : pos3[2]);
-            rope_sincos((float)pv * p.rope.freq[pair], sn, cs);
+          if (p.rope.axis[c * 16 + q] < 3) {
+            const float sn = (q & 1) ? sc[q >> 1].z : sc[q >> 1].x;
+            const float cs = (q & 1) ? sc[q >> 1].w : sc[q >> 1].y;
             const float a = v[2 * q], b = v[2 * q + 1];
             v[2 * q] = a * cs - b * sn;
             v[2 * q + 1] = a * sn + b * cs;
@@ -756,11 +771,21 @@ cudaError_t launch_pair_t(const GemmArgs& a, const CUtensorMap& ta, const CUtens
 
 }  // namespace
 
+cudaError_t launch_rope_table(const int32_t* pos, int64_t n, const RopeTable& rope, int pairs, float2* tab,
+                              cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  if (pairs < 1 || pairs > kMaxRopePairs || pos == nullptr || tab == nullptr) return cudaErrorInvalidValue;
+  const int64_t total = n * pairs;
+  rope_table_kernel<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(pos, n, rope, pairs, tab);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_gemm(const GemmArgs& a, PFN_cuTensorMapEncodeTiled_v12000 encode, int num_sms, cudaStream_t s) {
   if (a.M <= 0) return cudaSuccess;
   const int kb = a.int8 ? 128 : 64;
   if (a.K % kb != 0 || a.N % 128 != 0 || a.Nb % 128 != 0) return cudaErrorInvalidValue;
-  if (a.epi == kEpiQKV && (a.head_dim % 32 != 0 || (BN / 2) % a.head_dim != 0 || a.hd % a.head_dim != 0))
+  if (a.epi == kEpiQKV && (a.head_dim % 32 != 0 || (BN / 2) % a.head_dim != 0 || a.hd % a.head_dim != 0 ||
+                           a.rope_tab == nullptr || (reinterpret_cast<uintptr_t>(a.rope_tab) & 15) != 0))
     return cudaErrorInvalidValue;
   CUtensorMap ta, tb;
   if (make_map(encode, &ta, a.A, (uint64_t)a.M, (uint64_t)a.K, a.int8) != CUDA_SUCCESS) return cudaErrorInvalidValue;

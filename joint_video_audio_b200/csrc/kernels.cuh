@@ -97,10 +97,12 @@ struct GemmArgs {
   // kEpiQKV
   const __nv_bfloat16* q_gain;
   const __nv_bfloat16* k_gain;
-  const int32_t* pos;
   int head_dim, hd;
   float qk_eps;
   RopeTable rope;
+  // (sin, cos) of every rotary pair's angle per output row, [M, head_dim / 2]
+  // (launch_rope_table); required by kEpiQKV
+  const float2* rope_tab = nullptr;
   // kEpiStoreBf16: optional fp32 bias added per column
   const float* bias;
   // int8 dequantisation: acc * s_a[row] * s_b[col]
@@ -120,6 +122,14 @@ struct GemmArgs {
   int64_t ld_dump = 0;
 };
 cudaError_t launch_gemm(const GemmArgs& a, PFN_cuTensorMapEncodeTiled_v12000 encode, int num_sms, cudaStream_t s);
+
+// (sin, cos) of the rotary angle pos[row][axis(pair)] * freq[pair] for every
+// row and pair, tab[row * pairs + pair]; pairs without an axis get (0, 1).
+// Evaluated once per row here instead of once per query / key head in the
+// QKV epilogue, with the same reduction and hardware sine / cosine.
+cudaError_t launch_rope_table(const int32_t* pos, int64_t n, const RopeTable& rope, int pairs, float2* tab,
+                              cudaStream_t s);
+inline size_t rope_table_bytes(int64_t n, int pairs) { return (size_t)n * pairs * sizeof(float2); }
 
 // ---------------------------------------------------------------- attention
 struct AttnArgs {

@@ -30,7 +30,7 @@ using h3api::align256;
 using h3api::aligned16;
 
 struct ULayout {
-  size_t err, tiles, modt, h1, h1_q, h1_s, x1, h2, h2_q, h2_s, a, o_q, o_s, a_q, a_s, total;
+  size_t err, tiles, modt, rope, h1, h1_q, h1_s, x1, h2, h2_q, h2_s, a, o_q, o_s, a_q, a_s, total;
 };
 
 ULayout u_layout(const h3blk_config& c, int64_t n_total, int world) {
@@ -47,6 +47,7 @@ ULayout u_layout(const h3blk_config& c, int64_t n_total, int world) {
   L.err = put(4);
   L.tiles = put((size_t)((n_total + 127) / 128) * sizeof(h3::TileInfo));
   L.modt = put(q ? h3::modt_bytes(c.n_tags, c.n_t, c.hidden) : 0);
+  L.rope = put(h3::rope_table_bytes((int64_t)nl, c.head_dim / 2));
   if (q) {
     L.h1_q = put(nl * C);
     L.h1_s = put(nl * 4);
@@ -83,6 +84,7 @@ h3api::BlockBufs bufs(const h3blk_ctx* h, int64_t n_rows, const h3blk_ulysses* u
   b.err = reinterpret_cast<int*>(ws + L.err);
   b.tiles = reinterpret_cast<h3::TileInfo*>(ws + L.tiles);
   b.modt = reinterpret_cast<float4*>(ws + L.modt);
+  b.rope_tab = reinterpret_cast<float2*>(ws + L.rope);
   b.h1 = reinterpret_cast<__nv_bfloat16*>(at(L.h1, !q));
   b.h2 = reinterpret_cast<__nv_bfloat16*>(at(L.h2, !q));
   b.x1 = reinterpret_cast<__nv_bfloat16*>(ws + L.x1);

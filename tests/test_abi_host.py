@@ -82,9 +82,11 @@ def test_workspace_layout():
     n = 32768
     ws = blk.workspace_bytes(n)
     C_, HD, F = 5376, 7168, 14336
-    # h1, qkv, o, x1, h2, a in bf16
-    assert ws >= n * 2 * (C_ + 3 * HD + HD + C_ + C_ + F)
-    assert ws < n * 2 * (C_ + 3 * HD + HD + C_ + C_ + F) + 4 * 1024 * 1024
+    # h1, qkv, o, x1, h2, a in bf16, and the rotary (sin, cos) table: 64
+    # pairs x 8 bytes per row
+    stages = n * 2 * (C_ + 3 * HD + HD + C_ + C_ + F) + n * 64 * 8
+    assert ws >= stages
+    assert ws < stages + 4 * 1024 * 1024
     seen = []
     for name in ("ERROR", "H1", "QKV", "O", "X1", "H2", "A"):
         off, nb = B.h3blk_stage_view(blk.handle, n, name)
