@@ -37,6 +37,12 @@ sys.path.insert(0, ROOT)
 METRIC = "H3 block fwd packed rows/s @32k rows (bf16, W8A8) at 1 B200; % tensor peak"
 UNIT = "rows/s"
 PROFILES = os.path.join(ROOT, "profiles")
+# the library's kernel launches per block forward: tile summary, pre-norm,
+# rotary table, QKV GEMM, attention, out-projection GEMM, pre-norm, FFN up,
+# FFN down (bf16); W8A8 adds the modulation rearrangement and the two
+# standalone rotate + quantise passes; block-sparse adds pooling and selection
+LAUNCHES_BF16 = 9
+LAUNCHES_W8A8 = 12
 KERNEL_SOURCES = {  # interval name -> source file of its kernel (traffic records are tied to it)
     "attention": "joint_video_audio_b200/csrc/attn.cu",
     "qkv_gemm": "joint_video_audio_b200/csrc/gemm.cu",
@@ -344,7 +350,7 @@ def run_gpu_case(torch, j, hi, name, steps, warmup, device, peaks, int8_peak, cl
            "block_frac_of_ideal": ideal_s / (secs_max / steps),
            "value": aggregate_throughput(n, steps, int(os.environ.get("WORLD_SIZE", "1")), secs_max),
            "kernels": kernels, "roofline": roof, "clocks": clk,
-           "gpu_launches": steps * ((10 if dims.quant else 8) + (2 if density < 1.0 else 0))}
+           "gpu_launches": steps * (LAUNCHES_W8A8 if dims.quant else LAUNCHES_BF16) + steps * (2 if density < 1.0 else 0)}
     if density < 1.0:
         # work actually done: the kept (query tile, key tile) pairs
         lists = blk.stage(ws, n, "KV_LIST")
