@@ -96,6 +96,21 @@ def test_tiny_stage_qkv(tiny):
     assert_intermediate("v", v, ref["v"])
 
 
+def test_tiny_partial_rotary_split():
+    """Rotary pairs that follow no axis pass through unrotated (the page's own
+    split rotates 48 of 64 pairs at head_dim 128): 20 of 32 pairs rotated here,
+    the rest read (sin, cos) = (0, 1) from the table and are skipped."""
+    lay = hi.layout_tiny()
+    inp = hi.make_inputs(replace(hi.TINY, rope_pairs=(4, 8, 8)), lay)
+    case = GpuCase(inp)
+    case.run()
+    ref = orc.BlockOracle(inp.dims, inp.weights).forward(inp.x, lay.tag, lay.tidx, lay.pos, inp.table)
+    q, k, v = case.qkv()
+    assert_intermediate("q", q, ref["q"])
+    assert_intermediate("k", k, ref["k"])
+    assert_stage("out", case.out, ref["out"])
+
+
 def test_tiny_stage_attention(tiny):
     case, ref = tiny
     assert_intermediate("o", case.stage("O"), ref["o"])
