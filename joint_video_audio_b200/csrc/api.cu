@@ -186,9 +186,15 @@ namespace h3api {
 int check_block_weights(const h3blk_config& c, const h3blk_weights* w) {
   if (!w || !w->wqkv || !w->q_gain || !w->k_gain || !w->wo || !w->w13 || !w->w2) return H3BLK_ERR_INVALID_ARG;
   if (c.quant != 0 && (!w->s_qkv || !w->s_o || !w->s_13 || !w->s_2)) return H3BLK_ERR_INVALID_ARG;
-  const void* ptrs[] = {w->wqkv, w->wo, w->w13, w->w2};
+  // the GEMM epilogues read the gains and the int8 scales 16 bytes at a time
+  const void* ptrs[] = {w->wqkv, w->wo, w->w13, w->w2, w->q_gain, w->k_gain};
   for (const void* p : ptrs)
     if (!aligned16(p)) return H3BLK_ERR_INVALID_ARG;
+  if (c.quant != 0) {
+    const void* sc[] = {w->s_qkv, w->s_o, w->s_13, w->s_2};
+    for (const void* p : sc)
+      if (!aligned16(p)) return H3BLK_ERR_INVALID_ARG;
+  }
   return H3BLK_OK;
 }
 

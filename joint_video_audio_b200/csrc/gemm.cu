@@ -104,13 +104,6 @@ __device__ __forceinline__ void fail(const Smem& s, int* err) {
   *reinterpret_cast<volatile int*>(s.abort) = 1;
 }
 
-// fp32 value of accumulator register j of a chunk starting at column `col`
-template <bool INT8>
-__device__ __forceinline__ float acc_value(uint32_t r, float sa, const float* sb, int col) {
-  if (INT8) return (float)(int)r * sa * __ldg(sb + col);
-  return __uint_as_float(r);
-}
-
 __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&v)[32]) {
   uint4* d = reinterpret_cast<uint4*>(dst);
 #pragma unroll
@@ -134,8 +127,22 @@ __device__ __forceinline__ void load_chunk(uint32_t taddr, float sa, const float
 #pragma unroll
     for (int i = 0; i < 8; ++i) d[i] = make_uint4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
   }
+  if (INT8) {
+    // the chunk's 32 column scales, 16 bytes at a time (col is a multiple of
+    // 32 and the scale vectors are 16-byte aligned)
+    const float4* sb4 = reinterpret_cast<const float4*>(sb + col);
 #pragma unroll
-  for (int j = 0; j < 32; ++j) v[j] = acc_value<INT8>(r[j], sa, sb, col + j);
+    for (int i = 0; i < 8; ++i) {
+      const float4 b = __ldg(sb4 + i);
+      v[4 * i + 0] = (float)(int)r[4 * i + 0] * sa * b.x;
+      v[4 * i + 1] = (float)(int)r[4 * i + 1] * sa * b.y;
+      v[4 * i + 2] = (float)(int)r[4 * i + 2] * sa * b.z;
+      v[4 * i + 3] = (float)(int)r[4 * i + 3] * sa * b.w;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+  }
 }
 
 // cos and sin of a rotary angle: the angle is reduced to [-pi, pi] by a
@@ -305,8 +312,20 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tacc, 
         }
         float v[32];
         load_chunk<INT8>(th + c * 32, sa, p.s_b, col0 + c * 32, v, dump);
+        // the chunk's 32 gains, 16 bytes (8 bf16) at a time
+        const uint4* g4 = reinterpret_cast<const uint4*>(gain + c * 32);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = v[j] * rstd * __bfloat162float(gain[c * 32 + j]);
+        for (int i = 0; i < 4; ++i) {
+          const uint4 gw = __ldg(g4 + i);
+          const uint32_t gq[4] = {gw.x, gw.y, gw.z, gw.w};
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const float2 g2 = unpack_bf16x2(gq[h]);
+            const int j = 8 * i + 2 * h;
+            v[j] = v[j] * rstd * g2.x;
+            v[j + 1] = v[j + 1] * rstd * g2.y;
+          }
+        }
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
           if (p.rope.axis[c * 16 + q] < 3) {
