@@ -139,6 +139,23 @@ def test_forward_rejects_bad_arguments(override):
     assert _fake_forward(blk, 320, **override) == B.H3BLK_ERR_INVALID_ARG
 
 
+@pytest.mark.parametrize("field", ["q_gain", "k_gain"])
+def test_forward_rejects_misaligned_gains(field):
+    # the QKV epilogue reads the gains 16 bytes at a time; the check runs
+    # before any CUDA call, so the fake pointers are never dereferenced
+    blk = j.H3Block(hi.TINY)
+    n = 320
+    ws = blk.workspace_bytes(n)
+    base = 1 << 40
+    wd = dict(wqkv=base + (8 << 30), q_gain=base + (9 << 30), k_gain=base + (9 << 30) + 256,
+              wo=base + (10 << 30), w13=base + (11 << 30), w2=base + (12 << 30))
+    wd[field] += 8
+    w = B.h3blk_weights(**wd)
+    assert B.h3blk_forward(blk.handle, n, base, base + (1 << 30), base + (2 << 30), base + (3 << 30),
+                           base + (4 << 30), w, base + (5 << 30), base + (6 << 30), ws, None) == \
+        B.H3BLK_ERR_INVALID_ARG
+
+
 def test_forward_rejects_empty_sequence():
     blk = j.H3Block(hi.TINY)
     assert _fake_forward(blk, 0) == B.H3BLK_ERR_INVALID_ARG
