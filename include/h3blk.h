@@ -87,7 +87,9 @@ typedef struct {
 
 typedef struct h3blk_ctx* h3blk_handle;
 
-/* Weights of one block (device pointers, caller-owned).
+/* Weights of one block (device pointers, caller-owned, each 16-byte aligned:
+ * the GEMM epilogues read gains and scales 16 bytes at a time; a misaligned
+ * pointer is INVALID_ARG).
  * quant == 0: all matrices bf16; s_* unused (may be NULL).
  * quant == 1: matrices int8 as written by h3blk_prepare_int8_weights (input
  *             channels rotated by the block-128 Hadamard transform), s_* the
