@@ -167,8 +167,9 @@ def test_end_to_end_vs_oracle(name):
     ref["k"], ref["v"] = k_all[rows], v_all[rows]
     del k_all, v_all
     if dims.quant:
-        # int8 codes of the pre-attention norm (SURVEY reading c24: ties may
-        # round either way, so >= 99.9 % identical and never more than 1 apart)
+        # int8 codes of the pre-attention norm (a value within an ulp of a
+        # half-integer may round either way on the two sides, so >= 99.9 %
+        # identical and never more than 1 apart)
         q8 = _rows_gpu(case.stage("H1_Q8"), rows).cpu().numpy().astype(np.int64)
         rq, _ = orc.quantize_rows(orc.rotate_blocks(ref["h1"]))
         dq = np.abs(q8 - rq.astype(np.int64))

@@ -1,6 +1,6 @@
-"""The seeded synthetic workloads have the shapes the survey's input recipe
-states (row counts per modality, padding, tags, timestep indices, positions,
-dimensions), so every parity case and the bench run on the stated inputs."""
+"""The seeded synthetic workloads have the shapes their recipe states (row
+counts per modality, padding, tags, timestep indices, positions, dimensions),
+so every parity case and the bench run on the stated inputs."""
 import numpy as np
 import pytest
 
