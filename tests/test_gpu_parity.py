@@ -134,8 +134,9 @@ def test_tiny_stages_vs_faithful_oracle(tiny):
     """Against the oracle's diagnostic mode that rounds to bf16 where the GPU
     stores bf16 (h1, q, k, v, o, x1, a, out), h1 from the inputs and q, k, v
     from the GPU's h1: the fp32 arithmetic of the norm and of the QKV GEMM +
-    QK-norm + RoPE epilogue is off from fp64 by far less than one bf16 spacing of an O(1) value (fp32 sums of a few hundred products,
-    and the hardware sine / cosine at about 2^-21 absolute), so the stored
+    QK-norm + RoPE epilogue is off from fp64 by far less than one bf16
+    spacing of an O(1) value (fp32 sums of a few hundred products, and the
+    hardware sine / cosine at about 2^-21 absolute), so the stored
     h1, q, k and v can differ from the rounded fp64 values only where a value
     sits next to a rounding boundary: by at most one spacing plus that
     absolute error (which matters only for values near zero, where the
